@@ -1,0 +1,224 @@
+/*
+ * na2d_oracle.c -- plain, slow, fp64 reference for 2D Neighborhood Attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file; only the test suite, the smoke check and the CPU-baseline
+ * leg of the benchmark do.  It shares no code, header or table with the
+ * CUDA library.
+ *
+ * What it computes (Neighborhood Attention Transformer, Sec. 3.1, Eqs. (2)-(4),
+ * restated in the Qiita write-up "NAT: sliding-window attention", section
+ * "Neighborhood Attention (NA)"):
+ *
+ *   for every query pixel (i, j) of an H x W map, per batch b and head h,
+ *     A_n  = q(i,j) . key(r_n, t_n) + B(i,j ; r_n,t_n)                  Eq. (2)
+ *     V_n  = value(r_n, t_n)                                             Eq. (3)
+ *     out  = sum_n softmax(A / sqrt(d))_n * V_n                          Eq. (4)
+ *   over the ks x ks neighbourhood {(r_n, t_n)} of (i, j).
+ *
+ * Readings taken where the pages leave a step open:
+ *   - the neighbourhood is the ks x ks window whose start is
+ *     clamp(i - floor(ks/2), 0, H - ks) on rows (same on columns): every
+ *     pixel keeps the same span and corner pixels see a window that is not
+ *     centred on them (Sec. 1 and App. C "repeated windows at edge pixels";
+ *     the NA border drawing of the Qiita page);
+ *   - the bias B is read from a per-head (2ks-1) x (2ks-1) table at
+ *     [key_row - query_row + ks - 1][key_col - query_col + ks - 1];
+ *     a NULL table means zero bias (App. B.1 ablates the bias away);
+ *   - 1/sqrt(d) multiplies the bias as well as the dot product, exactly as
+ *     Eq. (4) divides the whole of A by sqrt(d); d is the per-head size;
+ *   - window entries are ordered row-major over the window: n = a*ks + c.
+ *
+ * Layouts (all contiguous, innermost last):
+ *   q, k, v, out : [B][heads][H][W][d]
+ *   rpb          : [heads][2ks-1][2ks-1]
+ *   attn         : [B][heads][H][W][ks*ks]
+ *
+ * All arithmetic is fp64.  Inputs that come from 16-bit tensors are
+ * converted exactly before they get here.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <stdint.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Start of the ks-wide window of position i on an axis of length L
+ * (Sec. 3.1 "nearest neighbours", App. C, Qiita NA border figure). */
+long na2d_oracle_window_start(long i, long L, long ks)
+{
+    long s = i - ks / 2;
+    if (s < 0) s = 0;
+    if (s > L - ks) s = L - ks;
+    return s;
+}
+
+static size_t idx5(long b, long h, long i, long j, long heads, long H, long W, long last)
+{
+    return ((((size_t)b * heads + h) * H + i) * W + j) * (size_t)last;
+}
+
+static double bias_at(const double *rpb, long h, long ks, long dr, long dc)
+{
+    long span = 2 * ks - 1;
+    if (!rpb) return 0.0;
+    return rpb[((size_t)h * span + (dr + ks - 1)) * span + (dc + ks - 1)];
+}
+
+/* Eq. (2) for one query: A[n] = q . key_n + B, unscaled. */
+static void logits_one(const double *q, const double *k, const double *rpb,
+                       long b, long h, long i, long j,
+                       long heads, long H, long W, long d, long ks, double *A)
+{
+    const double *qv = q + idx5(b, h, i, j, heads, H, W, d);
+    long si = na2d_oracle_window_start(i, H, ks);
+    long sj = na2d_oracle_window_start(j, W, ks);
+    for (long a = 0; a < ks; a++) {
+        for (long c = 0; c < ks; c++) {
+            long r = si + a, t = sj + c;
+            const double *kv = k + idx5(b, h, r, t, heads, H, W, d);
+            double dot = 0.0;
+            for (long x = 0; x < d; x++) dot += qv[x] * kv[x];
+            A[a * ks + c] = dot + bias_at(rpb, h, ks, r - i, t - j);
+        }
+    }
+}
+
+/* softmax(scale * A) over n entries, in place, with the maximum subtracted. */
+static void softmax_row(double *A, long n, double scale)
+{
+    double m = -INFINITY, sum = 0.0;
+    for (long t = 0; t < n; t++) if (scale * A[t] > m) m = scale * A[t];
+    for (long t = 0; t < n; t++) { A[t] = exp(scale * A[t] - m); sum += A[t]; }
+    for (long t = 0; t < n; t++) A[t] /= sum;
+}
+
+/* Eqs. (3)-(4) for one query: out = sum_n P[n] * value_n. */
+static void weighted_sum_one(const double *P, const double *v,
+                             long b, long h, long i, long j,
+                             long heads, long H, long W, long d, long ks, double *o)
+{
+    long si = na2d_oracle_window_start(i, H, ks);
+    long sj = na2d_oracle_window_start(j, W, ks);
+    for (long x = 0; x < d; x++) o[x] = 0.0;
+    for (long a = 0; a < ks; a++) {
+        for (long c = 0; c < ks; c++) {
+            const double *vv = v + idx5(b, h, si + a, sj + c, heads, H, W, d);
+            double p = P[a * ks + c];
+            for (long x = 0; x < d; x++) o[x] += p * vv[x];
+        }
+    }
+}
+
+static int threads_for(int nthreads)
+{
+#ifdef _OPENMP
+    return nthreads > 0 ? nthreads : omp_get_max_threads();
+#else
+    (void)nthreads;
+    return 1;
+#endif
+}
+
+/* The "QK + B" step alone (Eq. 2): attn = unscaled logits. */
+void na2d_oracle_qk_rpb(const double *q, const double *k, const double *rpb, double *attn,
+                        long B, long heads, long H, long W, long d, long ks, int nthreads)
+{
+    long rows = B * heads * H;
+#pragma omp parallel for schedule(dynamic) num_threads(threads_for(nthreads))
+    for (long row = 0; row < rows; row++) {
+        long i = row % H, bh = row / H, h = bh % heads, b = bh / heads;
+        for (long j = 0; j < W; j++)
+            logits_one(q, k, rpb, b, h, i, j, heads, H, W, d, ks,
+                       attn + idx5(b, h, i, j, heads, H, W, ks * ks));
+    }
+}
+
+/* softmax(scale * attn) over each row of ks*ks entries, in place (Eq. 4). */
+void na2d_oracle_softmax(double *attn, long nrows, long ks, double scale, int nthreads)
+{
+#pragma omp parallel for schedule(static) num_threads(threads_for(nthreads))
+    for (long r = 0; r < nrows; r++) softmax_row(attn + (size_t)r * ks * ks, ks * ks, scale);
+}
+
+/* The "AV" step alone (Eqs. 3-4): out = attn applied to the window's values. */
+void na2d_oracle_av(const double *attn, const double *v, double *out,
+                    long B, long heads, long H, long W, long d, long ks, int nthreads)
+{
+    long rows = B * heads * H;
+#pragma omp parallel for schedule(dynamic) num_threads(threads_for(nthreads))
+    for (long row = 0; row < rows; row++) {
+        long i = row % H, bh = row / H, h = bh % heads, b = bh / heads;
+        for (long j = 0; j < W; j++)
+            weighted_sum_one(attn + idx5(b, h, i, j, heads, H, W, ks * ks), v,
+                             b, h, i, j, heads, H, W, d, ks,
+                             out + idx5(b, h, i, j, heads, H, W, d));
+    }
+}
+
+/* Full NA_k (Eq. 4) for the rows row_begin <= (b*heads + h)*H + i < row_end
+ * (all W columns of each row); pass 0 and B*heads*H for the whole map. */
+void na2d_oracle_forward_rows(const double *q, const double *k, const double *v,
+                              const double *rpb, double *out,
+                              long B, long heads, long H, long W, long d, long ks,
+                              long row_begin, long row_end, int nthreads)
+{
+    double scale = 1.0 / sqrt((double)d);
+#pragma omp parallel num_threads(threads_for(nthreads))
+    {
+        double *A = (double *)malloc(sizeof(double) * (size_t)ks * ks);
+#pragma omp for schedule(dynamic)
+        for (long row = row_begin; row < row_end; row++) {
+            long i = row % H, bh = row / H, h = bh % heads, b = bh / heads;
+            for (long j = 0; j < W; j++) {
+                logits_one(q, k, rpb, b, h, i, j, heads, H, W, d, ks, A);
+                softmax_row(A, ks * ks, scale);
+                weighted_sum_one(A, v, b, h, i, j, heads, H, W, d, ks,
+                                 out + idx5(b, h, i, j, heads, H, W, d));
+            }
+        }
+        free(A);
+    }
+}
+
+void na2d_oracle_forward(const double *q, const double *k, const double *v,
+                         const double *rpb, double *out,
+                         long B, long heads, long H, long W, long d, long ks, int nthreads)
+{
+    na2d_oracle_forward_rows(q, k, v, rpb, out, B, heads, H, W, d, ks, 0, B * heads * H, nthreads);
+}
+
+/* Full NA_k for a list of n query points pts[4*t .. 4*t+3] = (b, h, i, j);
+ * out is [n][d] and, when attn is not NULL, the softmax weights go to
+ * attn [n][ks*ks] and the unscaled logits to logits [n][ks*ks] (either may be NULL). */
+void na2d_oracle_forward_points(const double *q, const double *k, const double *v,
+                                const double *rpb, const int64_t *pts, long n,
+                                double *out, double *logits, double *attn,
+                                long B, long heads, long H, long W, long d, long ks, int nthreads)
+{
+    double scale = 1.0 / sqrt((double)d);
+    (void)B;
+#pragma omp parallel num_threads(threads_for(nthreads))
+    {
+        double *A = (double *)malloc(sizeof(double) * (size_t)ks * ks);
+#pragma omp for schedule(dynamic)
+        for (long t = 0; t < n; t++) {
+            long b = (long)pts[4 * t], h = (long)pts[4 * t + 1];
+            long i = (long)pts[4 * t + 2], j = (long)pts[4 * t + 3];
+            logits_one(q, k, rpb, b, h, i, j, heads, H, W, d, ks, A);
+            if (logits)
+                for (long m = 0; m < ks * ks; m++) logits[(size_t)t * ks * ks + m] = A[m];
+            softmax_row(A, ks * ks, scale);
+            if (attn)
+                for (long m = 0; m < ks * ks; m++) attn[(size_t)t * ks * ks + m] = A[m];
+            weighted_sum_one(A, v, b, h, i, j, heads, H, W, d, ks, out + (size_t)t * d);
+        }
+        free(A);
+    }
+}
+
+int na2d_oracle_max_threads(void)
+{
+    return threads_for(0);
+}

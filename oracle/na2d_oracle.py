@@ -1,0 +1,205 @@
+"""ctypes front end of the fp64 C oracle (``na2d_oracle.c``).
+
+Test infrastructure only.  Arrays are numpy; everything is converted to
+contiguous float64 before the call, which is exact for fp32, fp16 and bf16
+values.  The shared object is compiled with gcc on first use (or by
+``build()``), next to the source.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "na2d_oracle.c")
+_LIB = os.path.join(_HERE, "libna2d_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_D = ctypes.POINTER(ctypes.c_double)
+_L = ctypes.c_long
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (plain -O2, IEEE arithmetic, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", tmp, _SRC, "-lm"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            lib.na2d_oracle_window_start.restype = _L
+            lib.na2d_oracle_window_start.argtypes = [_L, _L, _L]
+            lib.na2d_oracle_qk_rpb.argtypes = [_D, _D, _D, _D] + [_L] * 6 + [ctypes.c_int]
+            lib.na2d_oracle_softmax.argtypes = [_D, _L, _L, ctypes.c_double, ctypes.c_int]
+            lib.na2d_oracle_av.argtypes = [_D, _D, _D] + [_L] * 6 + [ctypes.c_int]
+            lib.na2d_oracle_forward.argtypes = [_D, _D, _D, _D, _D] + [_L] * 6 + [ctypes.c_int]
+            lib.na2d_oracle_forward_rows.argtypes = (
+                [_D, _D, _D, _D, _D] + [_L] * 6 + [_L, _L, ctypes.c_int]
+            )
+            lib.na2d_oracle_forward_points.argtypes = (
+                [_D, _D, _D, _D, ctypes.POINTER(ctypes.c_int64), _L, _D, _D, _D]
+                + [_L] * 6
+                + [ctypes.c_int]
+            )
+            lib.na2d_oracle_max_threads.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+class swapped_library:
+    """Context manager that points this module at another compiled copy of the
+    oracle (used by the test that plants mistakes in a copy of the source)."""
+
+    def __init__(self, path: str):
+        self.path = path
+
+    def __enter__(self):
+        global _lib
+        _load()
+        self._saved = _lib
+        lib = ctypes.CDLL(self.path)
+        for fn in ("na2d_oracle_window_start", "na2d_oracle_qk_rpb", "na2d_oracle_softmax",
+                   "na2d_oracle_av", "na2d_oracle_forward", "na2d_oracle_forward_rows",
+                   "na2d_oracle_forward_points", "na2d_oracle_max_threads"):
+            src, dst = getattr(self._saved, fn), getattr(lib, fn)
+            dst.argtypes, dst.restype = src.argtypes, src.restype
+        with _lock:
+            _lib = lib
+        return lib
+
+    def __exit__(self, *exc):
+        global _lib
+        with _lock:
+            _lib = self._saved
+        return False
+
+
+def compile_variant(source_text: str, out_path: str) -> str:
+    """Compiles a modified copy of the oracle source to out_path."""
+    src = out_path + ".c"
+    with open(src, "w") as f:
+        f.write(source_text)
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", out_path, src, "-lm"])
+    return out_path
+
+
+def source_text() -> str:
+    with open(_SRC) as f:
+        return f.read()
+
+
+def _f64(a):
+    if a is None:
+        return None
+    if hasattr(a, "detach"):  # a torch tensor: go through fp32, exact for 16-bit types
+        a = a.detach().cpu()
+        if a.dtype not in (_torch_f64(),):
+            a = a.float()
+        a = a.numpy()
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _torch_f64():
+    import torch
+
+    return torch.float64
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(_D)
+
+
+def _shape(q, ks):
+    B, heads, H, W, d = q.shape
+    if ks % 2 != 1 or ks < 1 or ks > H or ks > W:
+        raise ValueError(f"kernel size {ks} must be odd and fit the {H}x{W} map")
+    return B, heads, H, W, d
+
+
+def window_start(i: int, L: int, ks: int) -> int:
+    return int(_load().na2d_oracle_window_start(i, L, ks))
+
+
+def max_threads() -> int:
+    return int(_load().na2d_oracle_max_threads())
+
+
+def qk_rpb(q, k, rpb, ks: int, nthreads: int = 0) -> np.ndarray:
+    """Unscaled Eq. (2) logits, [B, heads, H, W, ks*ks]."""
+    q, k, rpb = _f64(q), _f64(k), _f64(rpb)
+    B, heads, H, W, d = _shape(q, ks)
+    attn = np.empty((B, heads, H, W, ks * ks), dtype=np.float64)
+    _load().na2d_oracle_qk_rpb(_ptr(q), _ptr(k), _ptr(rpb), _ptr(attn), B, heads, H, W, d, ks, nthreads)
+    return attn
+
+
+def softmax(attn, scale: float, nthreads: int = 0) -> np.ndarray:
+    """softmax(scale * attn) over the last axis (length ks*ks)."""
+    a = np.array(_f64(attn), dtype=np.float64, copy=True)
+    kk = a.shape[-1]
+    ks = int(round(kk ** 0.5))
+    assert ks * ks == kk
+    _load().na2d_oracle_softmax(_ptr(a), a.size // kk, ks, float(scale), nthreads)
+    return a
+
+
+def av(attn, v, ks: int, nthreads: int = 0) -> np.ndarray:
+    """Eqs. (3)-(4) with given weights: [B, heads, H, W, d]."""
+    attn, v = _f64(attn), _f64(v)
+    B, heads, H, W, d = _shape(v, ks)
+    out = np.empty_like(v)
+    _load().na2d_oracle_av(_ptr(attn), _ptr(v), _ptr(out), B, heads, H, W, d, ks, nthreads)
+    return out
+
+
+def forward(q, k, v, rpb, ks: int, nthreads: int = 0) -> np.ndarray:
+    """NA_k of Eq. (4) over the whole map: [B, heads, H, W, d]."""
+    q, k, v, rpb = _f64(q), _f64(k), _f64(v), _f64(rpb)
+    B, heads, H, W, d = _shape(q, ks)
+    out = np.empty_like(q)
+    _load().na2d_oracle_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(rpb), _ptr(out), B, heads, H, W, d, ks, nthreads)
+    return out
+
+
+def forward_rows(q, k, v, rpb, ks: int, row_begin: int, row_end: int, nthreads: int = 0) -> np.ndarray:
+    """NA_k for flattened rows [row_begin, row_end) of (b, h, i); returns the full-shape
+    output array with only those rows written (the rest is zero)."""
+    q, k, v, rpb = _f64(q), _f64(k), _f64(v), _f64(rpb)
+    B, heads, H, W, d = _shape(q, ks)
+    out = np.zeros_like(q)
+    _load().na2d_oracle_forward_rows(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(rpb), _ptr(out), B, heads, H, W, d, ks, row_begin, row_end, nthreads
+    )
+    return out
+
+
+def forward_points(q, k, v, rpb, ks: int, points, nthreads: int = 0):
+    """NA_k at the listed (b, h, i, j) points.
+
+    Returns (out [n, d], logits [n, ks*ks] unscaled, weights [n, ks*ks])."""
+    q, k, v, rpb = _f64(q), _f64(k), _f64(v), _f64(rpb)
+    B, heads, H, W, d = _shape(q, ks)
+    pts = np.ascontiguousarray(np.asarray(points, dtype=np.int64).reshape(-1, 4))
+    n = pts.shape[0]
+    out = np.empty((n, d), dtype=np.float64)
+    logits = np.empty((n, ks * ks), dtype=np.float64)
+    attn = np.empty((n, ks * ks), dtype=np.float64)
+    _load().na2d_oracle_forward_points(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(rpb),
+        pts.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n,
+        _ptr(out), _ptr(logits), _ptr(attn), B, heads, H, W, d, ks, nthreads,
+    )
+    return out, logits, attn

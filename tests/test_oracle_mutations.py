@@ -1,0 +1,64 @@
+"""Each plausible slip planted in a copy of the oracle source must make at
+least one pin of tests/test_oracle_pins.py fail.  The copies are compiled on
+the CPU into a temporary directory; the committed oracle is never changed."""
+import inspect
+
+import pytest
+
+import oracle
+from oracle import na2d_oracle as ora
+from tests import test_oracle_pins as pins
+
+MUTATIONS = {
+    "bias dropped": ("A[a * ks + c] = dot + bias_at(rpb, h, ks, r - i, t - j);",
+                     "A[a * ks + c] = dot;"),
+    "bias not divided by sqrt(d)": ("A[a * ks + c] = dot + bias_at(rpb, h, ks, r - i, t - j);",
+                                    "A[a * ks + c] = dot + sqrt((double)d) * bias_at(rpb, h, ks, r - i, t - j);"),
+    "bias rows and columns swapped": ("bias_at(rpb, h, ks, r - i, t - j)", "bias_at(rpb, h, ks, t - j, r - i)"),
+    "bias displacement sign flipped": ("bias_at(rpb, h, ks, r - i, t - j)", "bias_at(rpb, h, ks, i - r, j - t)"),
+    "window shifted by one": ("long s = i - ks / 2;", "long s = i - ks / 2 - 1;"),
+    "window clamped one short": ("if (s > L - ks) s = L - ks;", "if (s > L - ks) s = L - ks - (L > ks);"),
+    "keys used as values": ("weighted_sum_one(A, v,", "weighted_sum_one(A, k,"),
+    "no max subtraction": ("A[t] = exp(scale * A[t] - m);", "A[t] = exp(scale * A[t]);"),
+    "scale 1/d instead of 1/sqrt(d)": ("double scale = 1.0 / sqrt((double)d);\n#pragma omp parallel num_threads(threads_for(nthreads))\n    {\n        double *A = (double *)malloc(sizeof(double) * (size_t)ks * ks);\n#pragma omp for schedule(dynamic)\n        for (long row",
+                                       "double scale = 1.0 / (double)d;\n#pragma omp parallel num_threads(threads_for(nthreads))\n    {\n        double *A = (double *)malloc(sizeof(double) * (size_t)ks * ks);\n#pragma omp for schedule(dynamic)\n        for (long row"),
+    "window entries column-major": ("long r = si + a, t = sj + c;\n            const double *kv",
+                                    "long r = si + c, t = sj + a;\n            const double *kv"),
+    "column window sized by H": ("long sj = na2d_oracle_window_start(j, W, ks);\n    for (long a = 0; a < ks; a++) {\n        for (long c = 0; c < ks; c++) {\n            long r",
+                                 "long sj = na2d_oracle_window_start(j < H ? j : H - 1, H, ks);\n    for (long a = 0; a < ks; a++) {\n        for (long c = 0; c < ks; c++) {\n            long r"),
+}
+
+
+def _pin_cases():
+    """(name, callable) for every pin, with parametrized pins at each of their cases."""
+    cases = []
+    for name, fn in inspect.getmembers(pins, inspect.isfunction):
+        if not name.startswith("test_"):
+            continue
+        marks = getattr(fn, "pytestmark", [])
+        params = [m for m in marks if m.name == "parametrize"]
+        if not params:
+            cases.append((name, fn, {}))
+            continue
+        argnames, values = params[0].args
+        argnames = [a.strip() for a in argnames.split(",")] if isinstance(argnames, str) else list(argnames)
+        for val in values:
+            val = val if isinstance(val, tuple) else (val,)
+            cases.append((name, fn, dict(zip(argnames, val))))
+    return cases
+
+
+@pytest.mark.parametrize("mutation", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(mutation, tmp_path):
+    old, new = MUTATIONS[mutation]
+    text = ora.source_text()
+    assert text.count(old) >= 1, f"mutation anchor not found: {mutation}"
+    lib = ora.compile_variant(text.replace(old, new), str(tmp_path / "mutant.so"))
+    failed = []
+    with ora.swapped_library(lib):
+        for name, fn, kwargs in _pin_cases():
+            try:
+                fn(**kwargs)
+            except Exception:  # an assertion, or an error a pin provokes
+                failed.append(name)
+    assert failed, f"no pin caught the planted mistake: {mutation}"
