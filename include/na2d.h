@@ -1,0 +1,151 @@
+/*
+ * na2d.h -- C ABI of the B200 (sm_100a) 2D Neighborhood Attention library.
+ *
+ * The operator (Neighborhood Attention Transformer, Sec. 3.1, Eqs. (2)-(4);
+ * restated in the Qiita write-up "NAT: sliding-window attention", section
+ * "Neighborhood Attention (NA)"): for every query pixel (i, j) of an H x W
+ * map, per batch entry and head,
+ *
+ *   A_n    = q(i,j) . k(r_n,t_n) + B[h][r_n - i + ks - 1][t_n - j + ks - 1]   Eq. (2)
+ *   out    = sum_n softmax(A / sqrt(d))_n * v(r_n,t_n)                      Eqs. (3)-(4)
+ *
+ * over the ks x ks window r_n in [si, si+ks), t_n in [sj, sj+ks) with
+ * si = clamp(i - ks/2, 0, H - ks) and sj = clamp(j - ks/2, 0, W - ks)
+ * (Sec. 1 and App. C: every pixel keeps the same span, corner pixels get a
+ * window that is not centred on them).  The scale 1/sqrt(d) applies to the
+ * bias too, as Eq. (4) divides all of A.  Window entries are numbered
+ * row-major, n = a*ks + c for key (si + a, sj + c).
+ *
+ * Layouts (contiguous, C order, innermost last):
+ *   q, k, v, out : [B][heads][H][W][d]      element type given by na_dtype
+ *   rpb          : [heads][2*ks-1][2*ks-1]  same element type as q; may be NULL (zero bias,
+ *                                           the "no RPB" setting of App. B.1)
+ *   attn         : [B][heads][H][W][ks*ks]  always float32
+ *
+ * Ownership: the caller allocates and owns every buffer.  Device pointers
+ * must point to device memory of the current CUDA device and be 16-byte
+ * aligned.  The library allocates no memory in any call; it keeps only a
+ * per-device status word (a static device variable) and encoded TMA
+ * descriptors passed by value to its kernels.
+ *
+ * Streams: every call that takes `stream` (a cudaStream_t passed as void*,
+ * NULL meaning the legacy default stream) only enqueues work on it and
+ * returns; results are ready once the stream has been synchronised.
+ *
+ * Errors: argument errors are detected on the host before anything is
+ * enqueued and returned synchronously (NA_ERR_INVALID_ARG); shapes the
+ * library does not handle return NA_ERR_UNSUPPORTED; a failed launch or
+ * copy returns NA_ERR_CUDA.  Kernels never trap: a device-side wait that
+ * exceeds its time limit records NA_ERR_DEVICE_TIMEOUT in the status word,
+ * the kernel cleans up and returns, and na2d_device_status() reports it.
+ */
+#ifndef NA2D_H
+#define NA2D_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NA_OK = 0,
+    NA_ERR_INVALID_ARG = 1,
+    NA_ERR_UNSUPPORTED = 2,
+    NA_ERR_CUDA = 3,
+    NA_ERR_DEVICE_TIMEOUT = 4
+} na_status;
+
+typedef enum { NA_F32 = 0, NA_F16 = 1, NA_BF16 = 2 } na_dtype;
+
+/* Argument rules shared by the calls below: B >= 0 and heads >= 0 (either 0
+ * is an empty batch and a no-op); H, W >= 1; d in {16, 32, 64, 128}; ksize odd,
+ * 1 <= ksize <= min(H, W, 63); B*heads*H*W*max(d, ksize^2) < 2^62. */
+
+/*
+ * QK + B -- Eq. (2), the "QK+RPB" step of NATTEN (NAT paper Sec. 3.2;
+ * Qiita section "NATTEN": the library computes QK+B and AV separately).
+ * Writes the UNSCALED logits A (bias included, not divided by sqrt(d)) as
+ * float32 to attn [B][heads][H][W][ks*ks].  q, k, rpb are read-only.
+ */
+na_status na2d_qk_rpb(const void *q, const void *k, const void *rpb, float *attn,
+                      int B, int heads, int H, int W, int d, int ksize,
+                      na_dtype dt, void *stream);
+
+/*
+ * Softmax of Eq. (4), in place: each row of ksize*ksize entries of attn
+ * [B][heads][H][W][ks*ks] becomes softmax(scale * row) (the maximum is
+ * subtracted first).  Call with scale = 1/sqrt(d) between na2d_qk_rpb and
+ * na2d_av to obtain Eq. (4).
+ */
+na_status na2d_softmax(float *attn, int B, int heads, int H, int W, int ksize,
+                       float scale, void *stream);
+
+/*
+ * AV -- Eqs. (3)-(4) with given weights: out(i,j) = sum_n attn[i][j][n] * v(r_n, t_n),
+ * attn float32 [B][heads][H][W][ks*ks], v and out [B][heads][H][W][d] of type dt.
+ * Accumulates in float32 (float64 for NA_F32) and rounds to dt (nearest-even).
+ */
+na_status na2d_av(const float *attn, const void *v, void *out,
+                  int B, int heads, int H, int W, int d, int ksize,
+                  na_dtype dt, void *stream);
+
+/*
+ * Fused NA forward -- Eqs. (2)-(4) in one pass, out = NA_ks(q, k, v, rpb).
+ * fp16/bf16: tensor-core (tcgen05) logits and weighted sum with float32
+ * accumulation, softmax in float32, probabilities rounded to dt for the
+ * weighted sum, output rounded to dt.  fp32: float64 accumulation, output
+ * rounded to float32.  Nothing is materialised in global memory but out.
+ */
+na_status na2d_forward(const void *q, const void *k, const void *v, const void *rpb, void *out,
+                       int B, int heads, int H, int W, int d, int ksize,
+                       na_dtype dt, void *stream);
+
+/*
+ * na2d_forward from HOST buffers: copies q, k, v (and rpb when not NULL)
+ * host-to-device into the caller's device workspace, runs na2d_forward and
+ * copies the result back to out_host, all enqueued on `stream` (one
+ * cudaMemcpyAsync per buffer).  Pinned host memory makes the copies
+ * asynchronous; the host buffers must stay valid until the stream is
+ * synchronised.  workspace must be a 256-byte aligned device buffer of at
+ * least na2d_forward_host_workspace_bytes() bytes.
+ */
+size_t na2d_forward_host_workspace_bytes(int B, int heads, int H, int W, int d, int ksize,
+                                         na_dtype dt);
+na_status na2d_forward_host(const void *q_host, const void *k_host, const void *v_host,
+                            const void *rpb_host, void *out_host,
+                            void *workspace, size_t workspace_bytes,
+                            int B, int heads, int H, int W, int d, int ksize,
+                            na_dtype dt, void *stream);
+
+/*
+ * Which kernel na2d_forward launches for these arguments: 1 = tensor-core
+ * (tcgen05/TMEM/TMA) kernel, 0 = SIMT kernel, negative = the arguments are
+ * rejected (the negated na_status).  Host-only; enqueues nothing.
+ */
+int na2d_forward_kernel(int B, int heads, int H, int W, int d, int ksize, na_dtype dt);
+
+/*
+ * Synchronises `stream`, then returns and clears the status word of the
+ * current device: NA_ERR_DEVICE_TIMEOUT if any kernel gave up on a bounded
+ * wait since the last call, NA_ERR_CUDA if the stream reports a CUDA error,
+ * NA_OK otherwise.
+ */
+na_status na2d_device_status(void *stream);
+
+/*
+ * Test hook for the failure path: enqueues one kernel that waits on a
+ * barrier nothing ever releases, with a wait limit of timeout_us
+ * microseconds (1 .. 10^6).  The wait runs out, the kernel records
+ * NA_ERR_DEVICE_TIMEOUT and returns; the context stays usable.
+ */
+na_status na2d_debug_timeout_probe(unsigned int timeout_us, void *stream);
+
+/* Human-readable name of a status code (static string). */
+const char *na_status_str(na_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NA2D_H */

@@ -1,0 +1,247 @@
+// na2d_api.cu -- the extern "C" entry points of include/na2d.h: argument
+// checks, kernel selection, the per-device status word, the host-buffer
+// variant of the forward pass and the wait-timeout probe.
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "na2d_common.cuh"
+#include "na2d_internal.h"
+
+#define NA_EXPORT extern "C" __attribute__((visibility("default")))
+
+namespace na2d {
+namespace {
+
+// Status word of the device, written by kernels whose bounded waits ran
+// out; read and cleared by na2d_device_status().
+__device__ unsigned int g_status_word;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+unsigned* g_status_ptr[kMaxDevices] = {};
+
+// Device address of the status word on the current device (looked up once
+// per device with that device current).
+cudaError_t status_ptr(unsigned** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_status_word);
+    if (e != cudaSuccess) return e;
+    g_status_ptr[dev] = static_cast<unsigned*>(p);
+  }
+  *out = g_status_ptr[dev];
+  return cudaSuccess;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+na_status check_shape(int B, int heads, int H, int W, int d, int ks, bool need_d, Shape* s) {
+  if (B < 0 || heads < 0 || H < 1 || W < 1) return NA_ERR_INVALID_ARG;
+  if (ks < 1 || (ks & 1) == 0 || ks > H || ks > W || ks > 63) return NA_ERR_INVALID_ARG;
+  if (need_d && d != 16 && d != 32 && d != 64 && d != 128) return NA_ERR_INVALID_ARG;
+  const long double n = (long double)B * heads * H * W;
+  const long double per = (long double)(need_d ? (d > ks * ks ? d : ks * ks) : ks * ks);
+  if (n * per >= (long double)(1ll << 62)) return NA_ERR_INVALID_ARG;
+  *s = Shape{B, heads, H, W, need_d ? d : 0, ks};
+  return NA_OK;
+}
+
+na_status check_dtype(na_dtype dt) {
+  return (dt == NA_F32 || dt == NA_F16 || dt == NA_BF16) ? NA_OK : NA_ERR_INVALID_ARG;
+}
+
+size_t elem_size(na_dtype dt) { return dt == NA_F32 ? 4 : 2; }
+
+na_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NA_OK : NA_ERR_CUDA; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Which forward kernel runs (shape already validated).
+int forward_kernel_for(const Shape& s, na_dtype dt) {
+  return forward_tc_supported(s, dt) ? 1 : 0;
+}
+
+__global__ void timeout_probe_kernel(unsigned* status, unsigned long long limit_ns) {
+  __shared__ __align__(8) unsigned long long bar;
+  const unsigned addr = (unsigned)__cvta_generic_to_shared(&bar);
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(addr));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  // Nothing ever arrives on `bar`: this wait can only end by its limit.
+  const unsigned long long t0 = globaltimer_ns();
+  unsigned done = 0;
+  while (!done) {
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(addr), "r"(0u)
+        : "memory");
+    if (!done && globaltimer_ns() - t0 > limit_ns) {
+      atomicOr(status, kStatusTimeout);
+      break;
+    }
+  }
+}
+
+}  // namespace
+}  // namespace na2d
+
+using namespace na2d;
+
+NA_EXPORT const char* na_status_str(na_status s) {
+  switch (s) {
+    case NA_OK: return "NA_OK";
+    case NA_ERR_INVALID_ARG: return "NA_ERR_INVALID_ARG";
+    case NA_ERR_UNSUPPORTED: return "NA_ERR_UNSUPPORTED";
+    case NA_ERR_CUDA: return "NA_ERR_CUDA";
+    case NA_ERR_DEVICE_TIMEOUT: return "NA_ERR_DEVICE_TIMEOUT";
+  }
+  return "NA_ERR_UNKNOWN";
+}
+
+NA_EXPORT na_status na2d_qk_rpb(const void* q, const void* k, const void* rpb, float* attn,
+                                int B, int heads, int H, int W, int d, int ksize, na_dtype dt,
+                                void* stream) {
+  Shape s;
+  na_status st = check_dtype(dt);
+  if (st == NA_OK) st = check_shape(B, heads, H, W, d, ksize, true, &s);
+  if (st != NA_OK) return st;
+  if (!q || !k || !attn || !aligned16(q) || !aligned16(k) || !aligned16(attn)) return NA_ERR_INVALID_ARG;
+  if (rpb && !aligned16(rpb)) return NA_ERR_INVALID_ARG;
+  if (s.queries() == 0) return NA_OK;
+  return from_cuda(launch_qk_rpb_simt(q, k, rpb, attn, s, dt, (cudaStream_t)stream));
+}
+
+NA_EXPORT na_status na2d_softmax(float* attn, int B, int heads, int H, int W, int ksize,
+                                 float scale, void* stream) {
+  Shape s;
+  na_status st = check_shape(B, heads, H, W, 0, ksize, false, &s);
+  if (st != NA_OK) return st;
+  if (!attn || !aligned16(attn) || !std::isfinite(scale)) return NA_ERR_INVALID_ARG;
+  if (s.queries() == 0) return NA_OK;
+  return from_cuda(launch_softmax_simt(attn, s.queries(), ksize, scale, (cudaStream_t)stream));
+}
+
+NA_EXPORT na_status na2d_av(const float* attn, const void* v, void* out, int B, int heads, int H,
+                            int W, int d, int ksize, na_dtype dt, void* stream) {
+  Shape s;
+  na_status st = check_dtype(dt);
+  if (st == NA_OK) st = check_shape(B, heads, H, W, d, ksize, true, &s);
+  if (st != NA_OK) return st;
+  if (!attn || !v || !out || !aligned16(attn) || !aligned16(v) || !aligned16(out)) return NA_ERR_INVALID_ARG;
+  if (s.queries() == 0) return NA_OK;
+  return from_cuda(launch_av_simt(attn, v, out, s, dt, (cudaStream_t)stream));
+}
+
+NA_EXPORT int na2d_forward_kernel(int B, int heads, int H, int W, int d, int ksize, na_dtype dt) {
+  Shape s;
+  na_status st = check_dtype(dt);
+  if (st == NA_OK) st = check_shape(B, heads, H, W, d, ksize, true, &s);
+  if (st != NA_OK) return -(int)st;
+  return forward_kernel_for(s, dt);
+}
+
+NA_EXPORT na_status na2d_forward(const void* q, const void* k, const void* v, const void* rpb,
+                                 void* out, int B, int heads, int H, int W, int d, int ksize,
+                                 na_dtype dt, void* stream) {
+  Shape s;
+  na_status st = check_dtype(dt);
+  if (st == NA_OK) st = check_shape(B, heads, H, W, d, ksize, true, &s);
+  if (st != NA_OK) return st;
+  if (!q || !k || !v || !out) return NA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return NA_ERR_INVALID_ARG;
+  if (rpb && !aligned16(rpb)) return NA_ERR_INVALID_ARG;
+  if (s.queries() == 0) return NA_OK;
+  cudaStream_t cs = (cudaStream_t)stream;
+  if (forward_kernel_for(s, dt) == 1) {
+    unsigned* status = nullptr;
+    cudaError_t e = status_ptr(&status);
+    if (e != cudaSuccess) return NA_ERR_CUDA;
+    return from_cuda(launch_forward_tc(q, k, v, rpb, out, s, dt, status, cs));
+  }
+  return from_cuda(launch_forward_simt(q, k, v, rpb, out, s, dt, cs));
+}
+
+namespace {
+struct HostLayout {
+  size_t q, k, v, rpb, out, total, tensor_bytes, rpb_bytes;
+};
+// The workspace always reserves room for the bias table, so its size does
+// not depend on whether the caller passes one.
+HostLayout host_layout(const Shape& s, na_dtype dt) {
+  HostLayout L{};
+  const size_t es = elem_size(dt);
+  L.tensor_bytes = (size_t)s.queries() * (size_t)s.d * es;
+  L.rpb_bytes = (size_t)s.heads * (2 * s.ks - 1) * (2 * s.ks - 1) * es;
+  size_t off = 0;
+  L.q = off; off = round_up(off + L.tensor_bytes, 256);
+  L.k = off; off = round_up(off + L.tensor_bytes, 256);
+  L.v = off; off = round_up(off + L.tensor_bytes, 256);
+  L.out = off; off = round_up(off + L.tensor_bytes, 256);
+  L.rpb = off; off = round_up(off + L.rpb_bytes, 256);
+  L.total = off;
+  return L;
+}
+}  // namespace
+
+NA_EXPORT size_t na2d_forward_host_workspace_bytes(int B, int heads, int H, int W, int d, int ksize,
+                                                   na_dtype dt) {
+  Shape s;
+  if (check_dtype(dt) != NA_OK || check_shape(B, heads, H, W, d, ksize, true, &s) != NA_OK) return 0;
+  return host_layout(s, dt).total;
+}
+
+NA_EXPORT na_status na2d_forward_host(const void* q_host, const void* k_host, const void* v_host,
+                                      const void* rpb_host, void* out_host, void* workspace,
+                                      size_t workspace_bytes, int B, int heads, int H, int W, int d,
+                                      int ksize, na_dtype dt, void* stream) {
+  Shape s;
+  na_status st = check_dtype(dt);
+  if (st == NA_OK) st = check_shape(B, heads, H, W, d, ksize, true, &s);
+  if (st != NA_OK) return st;
+  if (!q_host || !k_host || !v_host || !out_host || !workspace) return NA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NA_ERR_INVALID_ARG;
+  const HostLayout L = host_layout(s, dt);
+  if (workspace_bytes < L.total) return NA_ERR_INVALID_ARG;
+  if (s.queries() == 0) return NA_OK;
+  cudaStream_t cs = (cudaStream_t)stream;
+  char* ws = static_cast<char*>(workspace);
+  cudaError_t e = cudaMemcpyAsync(ws + L.q, q_host, L.tensor_bytes, cudaMemcpyHostToDevice, cs);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(ws + L.k, k_host, L.tensor_bytes, cudaMemcpyHostToDevice, cs);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(ws + L.v, v_host, L.tensor_bytes, cudaMemcpyHostToDevice, cs);
+  if (e == cudaSuccess && rpb_host)
+    e = cudaMemcpyAsync(ws + L.rpb, rpb_host, L.rpb_bytes, cudaMemcpyHostToDevice, cs);
+  if (e != cudaSuccess) return NA_ERR_CUDA;
+  st = na2d_forward(ws + L.q, ws + L.k, ws + L.v, rpb_host ? ws + L.rpb : nullptr, ws + L.out, B, heads,
+                    H, W, d, ksize, dt, stream);
+  if (st != NA_OK) return st;
+  return from_cuda(cudaMemcpyAsync(out_host, ws + L.out, L.tensor_bytes, cudaMemcpyDeviceToHost, cs));
+}
+
+NA_EXPORT na_status na2d_device_status(void* stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return NA_ERR_CUDA;
+  unsigned* p = nullptr;
+  if (status_ptr(&p) != cudaSuccess) return NA_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpy(&v, p, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return NA_ERR_CUDA;
+  if (v && cudaMemset(p, 0, sizeof(v)) != cudaSuccess) return NA_ERR_CUDA;
+  return (v & kStatusTimeout) ? NA_ERR_DEVICE_TIMEOUT : NA_OK;
+}
+
+NA_EXPORT na_status na2d_debug_timeout_probe(unsigned int timeout_us, void* stream) {
+  if (timeout_us < 1 || timeout_us > 1000000u) return NA_ERR_INVALID_ARG;
+  unsigned* p = nullptr;
+  if (status_ptr(&p) != cudaSuccess) return NA_ERR_CUDA;
+  timeout_probe_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(p, 1000ull * timeout_us);
+  return from_cuda(cudaGetLastError());
+}
