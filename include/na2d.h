@@ -32,6 +32,9 @@
  * NULL meaning the legacy default stream) only enqueues work on it and
  * returns; results are ready once the stream has been synchronised.
  *
+ * An empty batch (B == 0 or heads == 0) is a no-op that returns NA_OK
+ * without looking at the buffer pointers (they may be NULL).
+ *
  * Errors: argument errors are detected on the host before anything is
  * enqueued and returned synchronously (NA_ERR_INVALID_ARG); shapes the
  * library does not handle return NA_ERR_UNSUPPORTED; a failed launch or

@@ -116,9 +116,9 @@ NA_EXPORT na_status na2d_qk_rpb(const void* q, const void* k, const void* rpb, f
   na_status st = check_dtype(dt);
   if (st == NA_OK) st = check_shape(B, heads, H, W, d, ksize, true, &s);
   if (st != NA_OK) return st;
+  if (s.queries() == 0) return NA_OK;  // empty batch: nothing is read or written
   if (!q || !k || !attn || !aligned16(q) || !aligned16(k) || !aligned16(attn)) return NA_ERR_INVALID_ARG;
   if (rpb && !aligned16(rpb)) return NA_ERR_INVALID_ARG;
-  if (s.queries() == 0) return NA_OK;
   return from_cuda(launch_qk_rpb_simt(q, k, rpb, attn, s, dt, (cudaStream_t)stream));
 }
 
@@ -127,8 +127,9 @@ NA_EXPORT na_status na2d_softmax(float* attn, int B, int heads, int H, int W, in
   Shape s;
   na_status st = check_shape(B, heads, H, W, 0, ksize, false, &s);
   if (st != NA_OK) return st;
-  if (!attn || !aligned16(attn) || !std::isfinite(scale)) return NA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return NA_ERR_INVALID_ARG;
   if (s.queries() == 0) return NA_OK;
+  if (!attn || !aligned16(attn)) return NA_ERR_INVALID_ARG;
   return from_cuda(launch_softmax_simt(attn, s.queries(), ksize, scale, (cudaStream_t)stream));
 }
 
@@ -138,8 +139,8 @@ NA_EXPORT na_status na2d_av(const float* attn, const void* v, void* out, int B, 
   na_status st = check_dtype(dt);
   if (st == NA_OK) st = check_shape(B, heads, H, W, d, ksize, true, &s);
   if (st != NA_OK) return st;
-  if (!attn || !v || !out || !aligned16(attn) || !aligned16(v) || !aligned16(out)) return NA_ERR_INVALID_ARG;
   if (s.queries() == 0) return NA_OK;
+  if (!attn || !v || !out || !aligned16(attn) || !aligned16(v) || !aligned16(out)) return NA_ERR_INVALID_ARG;
   return from_cuda(launch_av_simt(attn, v, out, s, dt, (cudaStream_t)stream));
 }
 
@@ -158,10 +159,10 @@ NA_EXPORT na_status na2d_forward(const void* q, const void* k, const void* v, co
   na_status st = check_dtype(dt);
   if (st == NA_OK) st = check_shape(B, heads, H, W, d, ksize, true, &s);
   if (st != NA_OK) return st;
+  if (s.queries() == 0) return NA_OK;
   if (!q || !k || !v || !out) return NA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return NA_ERR_INVALID_ARG;
   if (rpb && !aligned16(rpb)) return NA_ERR_INVALID_ARG;
-  if (s.queries() == 0) return NA_OK;
   cudaStream_t cs = (cudaStream_t)stream;
   if (forward_kernel_for(s, dt) == 1) {
     unsigned* status = nullptr;
@@ -209,11 +210,11 @@ NA_EXPORT na_status na2d_forward_host(const void* q_host, const void* k_host, co
   na_status st = check_dtype(dt);
   if (st == NA_OK) st = check_shape(B, heads, H, W, d, ksize, true, &s);
   if (st != NA_OK) return st;
+  if (s.queries() == 0) return NA_OK;
   if (!q_host || !k_host || !v_host || !out_host || !workspace) return NA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NA_ERR_INVALID_ARG;
   const HostLayout L = host_layout(s, dt);
   if (workspace_bytes < L.total) return NA_ERR_INVALID_ARG;
-  if (s.queries() == 0) return NA_OK;
   cudaStream_t cs = (cudaStream_t)stream;
   char* ws = static_cast<char*>(workspace);
   cudaError_t e = cudaMemcpyAsync(ws + L.q, q_host, L.tensor_bytes, cudaMemcpyHostToDevice, cs);
