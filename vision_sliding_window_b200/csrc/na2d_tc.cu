@@ -1,27 +1,33 @@
 // na2d_tc.cu -- tensor-core fused forward of 2D Neighborhood Attention for
 // fp16 / bf16 on sm_100a (Neighborhood Attention Transformer, Sec. 3.1,
-// Eqs. (2)-(4); the tiling follows the "tiled NA" idea of Sec. 3.2 and
-// App. A.4: a query tile plus its key/value halo staged in shared memory).
+// Eqs. (2)-(4)).  The data movement follows the "tiled NA" idea of Sec. 3.2
+// and App. A.4 -- a query tile plus the key/value halo its windows cover,
+// staged in shared memory -- re-planned for TMA, tcgen05 and tensor memory.
 //
-// One persistent CTA per SM walks a list of 8 x 16 query tiles.  Per tile:
-//   * TMA loads the query tile (four 4 x 8 patches) and the K and V halo --
-//     the (8+k-1) x (16+k-1, rounded up to 8) keys every window of the tile
-//     lies in -- into swizzled shared memory (double-buffered).
-//   * One thread issues tcgen05.mma: S = Q_tile . K_halo^T (M = 128 queries,
-//     N = halo keys, float32 in tensor memory).
-//   * Four softmax warps, each owning one 4 x 8 patch (32 TMEM lanes), read
-//     only the union of their 32 windows from tensor memory, add the bias
-//     (and -inf outside each query's clamped window) from a per-head table in
-//     shared memory, take the row maximum, then write exp2((s - m) * log2e /
-//     sqrt(d)) rounded to 16 bits back over S as the P operand (zeros outside
-//     the union).
-//   * tcgen05.mma: O = P . V_halo (A = P from tensor memory, B = V in shared
-//     memory, N = d), then the softmax warps divide by the row sum and store.
+// Work unit: a "pair" of 8x8 query tiles stacked vertically (16 x 8
+// queries).  Each tile is one M = 64 MMA; tile A writes tensor-memory lanes
+// 0-15 of every 32-lane quarter, tile B lanes 16-31, so the two share the
+// same columns.  The pair's K and V halo -- (16+k-1) rows x (8+k-1, rounded
+// up to 8) columns -- is one TMA box each; tile B's halo starts 8 rows
+// further down inside the same buffer.
+//
+// Roles of one persistent CTA per SM:
+//   warp 0      TMA producer (query patches, K halo, V halo; STAGES buffers)
+//   warp 1      tensor-memory allocation; one lane issues every tcgen05.mma
+//   warps 2..   NBUF softmax warpgroups; group g owns tensor-memory buffer g
+//               and every NBUF-th pair, so one group's P.V and epilogue
+//               overlap the other group's softmax.
+// Per pair:  S = Q K_halo^T (fp32, tensor memory) -> each softmax warp reads
+// the union of the windows of its two 4x4 patches (one per tile), adds the
+// bias and the -inf mask from a per-head table, keeps x = s + bias in place,
+// takes the row maximum, then writes P = exp2((x - max) log2e / sqrt(d)) in
+// 16 bits over S (zeros outside the union) -> O = P V_halo -> O / rowsum.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include <cmath>
 #include <mutex>
+#include <type_traits>
 
 #include "na2d_common.cuh"
 #include "na2d_internal.h"
@@ -32,73 +38,88 @@ namespace {
 
 using namespace sm100;
 
-constexpr int TH = 8, TW = 16;  // query tile (rows x columns), 128 queries = MMA M
-constexpr int PH = 4, PW = 8;   // query patch of one softmax warp (32 TMEM lanes)
-constexpr int kSoftmaxWarps = 4;
-constexpr int kThreads = 32 * (2 + kSoftmaxWarps);
+constexpr int TT = 8;  // 8 x 8 query tile
+constexpr int PQ = 4;  // 4 x 4 patch: the 16 lanes of one tile a softmax warp owns
 constexpr int kTmemCols = 512;
-constexpr int kMinSmem = 116 * 1024;  // keeps one CTA per SM (it holds all of tensor memory)
+constexpr int kMaxSmem = 227 * 1024;
+constexpr int kMinSmem = 116 * 1024;  // one CTA per SM: it holds all of tensor memory
+
+__host__ __device__ constexpr int round_up(int x, int a) { return (x + a - 1) / a * a; }
 
 template <int KS, int D>
 struct Cfg {
-  static constexpr int HH = TH + KS - 1;                    // halo rows
-  static constexpr int HW = (TW + KS - 1 + 7) / 8 * 8;      // halo columns, multiple of 8
-  static constexpr int NS = HH * HW;                        // halo keys = S columns
-  static constexpr int NP = HW / 8;                         // 8-key pieces per halo row
-  static constexpr int ROWB = D * 2;                        // bytes per key / query row
-  static constexpr int Q_BYTES = TH * TW * ROWB;
-  static constexpr int KV_BYTES = NS * ROWB;
+  static constexpr int HH = TT + KS - 1;               // halo rows of one tile
+  static constexpr int HHP = 2 * TT + KS - 1;          // halo rows of the pair buffer
+  static constexpr int HW = round_up(TT + KS - 1, 8);  // halo columns
+  static constexpr int NS = HH * HW;                   // keys of one tile = S columns
+  static constexpr int NPC = HW / 4;                   // 4-key pieces per halo row
+  static constexpr int NPU = (PQ - 1 + KS + 3) / 4;    // pieces of an interior patch's window union
+  static constexpr int ROWB = 2 * D;                   // bytes per key / query row
+  static constexpr int QBLK = 2 * TT * TT * ROWB;      // one K block of the query operand (128 rows)
+  static constexpr int Q_BYTES = 2 * QBLK;
+  static constexpr int KV_BYTES = HHP * HW * ROWB;
   static constexpr int STAGE_BYTES = Q_BYTES + 2 * KV_BYTES;
-  // bias / mask table: rows 0..2KS-2 are bias rows, row 2KS-1 is all -inf.
-  // Row layout: KS blocks of stride KS+PAD, block dc = [PAD x -inf][bias
-  // row, columns dc .. dc+KS-1][shared with the next block's -inf pad].
-  static constexpr int PAD = (PW - 1) + 7;
+  // tensor memory: per buffer S (NS columns); P (16-bit) overlays its first
+  // NS/2 columns; O (2d columns: tile A's d, then tile B's d) sits in the
+  // dead part of S after P.
+  static constexpr int NBUF = NS <= kTmemCols / 2 ? 2 : 1;
+  static constexpr int BUF_COLS = kTmemCols / NBUF;
+  static constexpr int PO = round_up(NS / 2, 32);
+  // bias / mask table (one per softmax group): rows 0..2KS-2 hold bias rows,
+  // row 2KS-1 is all -inf.  A row is KS blocks of stride KS+PAD; block dc
+  // holds the bias row's columns dc..dc+KS-1 after PAD entries of -inf, and
+  // its tail is the next block's -inf head.  PAD covers a whole halo row
+  // around any window.
+  static constexpr int PAD = HW - KS;
   static constexpr int TBL_W0 = KS * (KS + PAD) + PAD;
-  static constexpr int TBL_W = TBL_W0 + ((8 - TBL_W0 % 32) + 32) % 32;  // = 8 mod 32: no bank conflicts
+  static constexpr int TBL_W = TBL_W0 + ((8 - TBL_W0 % 32) + 32) % 32;  // = 8 mod 32: conflict-free rows
   static constexpr int TBL_ROWS = 2 * KS;
   static constexpr int TBL_BYTES = TBL_ROWS * TBL_W * 4;
-  static constexpr int STAGES = (2 * STAGE_BYTES + TBL_BYTES + 4096 <= 200 * 1024) ? 2 : 1;
-  static constexpr int S_COL = 0;
-  static constexpr int O_COL = (NS + 31) / 32 * 32;
-  static constexpr int SMEM_BYTES_RAW = 1024 + STAGES * STAGE_BYTES + TBL_BYTES + 256;
-  static constexpr int SMEM_BYTES = SMEM_BYTES_RAW > kMinSmem ? SMEM_BYTES_RAW : kMinSmem;
+  static constexpr int FIXED = 1024 + NBUF * TBL_BYTES + 512;
+  static constexpr int STAGES_FIT = (kMaxSmem - FIXED) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT >= 3 ? 3 : STAGES_FIT;
+  static constexpr int SMEM_RAW = FIXED + STAGES * STAGE_BYTES;
+  static constexpr int SMEM_BYTES = SMEM_RAW > kMinSmem ? SMEM_RAW : kMinSmem;
+  static constexpr int THREADS = 64 + 128 * NBUF;
   static constexpr uint32_t LAYOUT = ROWB == 64 ? kLayoutSW64 : kLayoutSW128;
-  static_assert(O_COL + D <= kTmemCols, "S and O must fit in tensor memory");
+  static_assert(NS <= BUF_COLS && PO + 2 * D <= BUF_COLS, "S, P and O of a buffer must fit in tensor memory");
+  static_assert(STAGES >= 1, "a pipeline stage must fit in shared memory");
   static_assert(NS % 16 == 0, "halo keys must be a multiple of the MMA K step");
-  static_assert(Q_BYTES % 1024 == 0 && KV_BYTES % 1024 == 0, "swizzle atoms must stay aligned");
-  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+  static_assert(QBLK % 1024 == 0 && KV_BYTES % 1024 == 0 && (TT * HW * ROWB) % 1024 == 0,
+                "swizzle atoms must stay aligned");
+  static_assert(SMEM_BYTES <= kMaxSmem, "shared memory");
 };
 
 struct Params {
   const void* rpb;  // [heads][2KS-1][2KS-1] or nullptr
   void* out;
   int B, heads, H, W;
-  int n_tr, n_tc, total_tiles;
-  float scale_log2;  // log2(e) / sqrt(d)
+  int n_pr, n_pc, total;  // pair rows / columns per map, pairs in all
+  float scale_log2;       // log2(e) / sqrt(d)
   unsigned* status;
 };
 
-struct Tile {
-  int b, h, i0, j0, r0, c0;
+// A pair of 8x8 tiles: rows [i0, i0+16), columns [j0, j0+8) of map (b, h).
+// Halo origin (R0, c0); tile B's windows start rB rows below R0.
+struct Pair {
+  int b, h, i0, j0, R0, c0, rB;
 };
 
 template <int KS>
-NA_DEVICE Tile decode_tile(int t, const Params& p) {
-  Tile tl;
-  const int tc = t % p.n_tc;
-  int rest = t / p.n_tc;
-  const int tr = rest % p.n_tr;
-  rest /= p.n_tr;
-  tl.b = rest % p.B;
-  tl.h = rest / p.B;
-  tl.i0 = tr * TH;
-  tl.j0 = tc * TW;
-  // Halo origin: every window of the tile's queries lies in
-  // [r0, r0 + HH) x [c0, c0 + HW); out-of-map parts are zero-filled by TMA.
-  tl.r0 = window_start(tl.i0, p.H, KS);
-  const int cj = window_start(tl.j0, p.W, KS);
-  tl.c0 = min(tl.j0 - KS / 2, cj);
-  return tl;
+NA_DEVICE Pair decode_pair(int t, const Params& p) {
+  Pair q;
+  const int pc = t % p.n_pc;
+  int rest = t / p.n_pc;
+  const int pr = rest % p.n_pr;
+  rest /= p.n_pr;
+  q.b = rest % p.B;
+  q.h = rest / p.B;
+  q.i0 = pr * 2 * TT;
+  q.j0 = pc * TT;
+  q.R0 = window_start(q.i0, p.H, KS);
+  q.rB = window_start(min(q.i0 + TT, p.H - 1), p.H, KS) - q.R0;  // 0 .. 8
+  q.c0 = min(q.j0 - KS / 2, window_start(q.j0, p.W, KS));
+  return q;
 }
 
 template <typename T> NA_DEVICE float to_f(T x);
@@ -115,37 +136,192 @@ template <> NA_DEVICE uint32_t pack2<__half>(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Stores N (a multiple of 4) consecutive 32-bit columns from registers.
+template <int N>
+NA_DEVICE void tmem_st_row(uint32_t taddr, const uint32_t (&r)[N]) {
+  static_assert(N % 4 == 0, "row stores go by 4 columns");
+#pragma unroll
+  for (int c = 0; c < N; c += 4) {
+    const uint32_t v[4] = {r[c], r[c + 1], r[c + 2], r[c + 3]};
+    tmem_st4(taddr + c, v);
+  }
+}
+
+// Loads pieces [PB, PB+NU) (4 columns each) of halo row `row` of S.
+template <int HW, int PB, int NU>
+NA_DEVICE void load_pieces(uint32_t row, uint32_t (&v)[NU * 4]) {
+  if constexpr (PB == 0 && NU * 4 == 16) {
+    tmem_ld16(row, v);
+  } else {
+#pragma unroll
+    for (int u = 0; u < NU; ++u) {
+      uint32_t w[4];
+      tmem_ld4(row + (PB + u) * 4, w);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[4 * u + e] = w[e];
+    }
+  }
+}
+
+// Softmax of one warp's 32 queries (two 4x4 patches) over the union rows
+// [u_r0, u_r1) and pieces [PB, PB+NU) of their windows.  Pass 1 writes
+// x = s + bias (-inf outside the window) back over S and takes the row
+// maximum; pass 2 writes P = exp2(x c - max c) as 16-bit pairs over S (P
+// row hr covers the S columns of row hr/2, which pass 2 has already read)
+// and returns the row sum.  Rows are processed two at a time with the next
+// row's loads in flight.
+template <typename T, int KS, int D, int PB, int NU>
+NA_DEVICE float softmax_rows(uint32_t sbuf, const float* tbl, int u_r0, int u_r1, int wr0, int er,
+                             int colbase, float c) {
+  using C = Cfg<KS, D>;
+  constexpr int NV = NU * 4;
+  auto trow_of = [&](int hr) {
+    return tbl + ((unsigned)(hr - wr0) < (unsigned)KS ? hr + er : 2 * KS - 1) * C::TBL_W + colbase + PB * 4;
+  };
+  float m0 = -INFINITY, m1 = -INFINITY;
+  auto bias_row = [&](int hr, uint32_t (&v)[NV]) {
+    const float* tr = trow_of(hr);
+#pragma unroll
+    for (int e = 0; e < NV; e += 4) {
+      float x0, x1, x2, x3;
+      add2(x0, x1, __uint_as_float(v[e]), __uint_as_float(v[e + 1]), tr[e], tr[e + 1]);
+      add2(x2, x3, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]), tr[e + 2], tr[e + 3]);
+      m0 = max3(m0, x0, x1);
+      m1 = max3(m1, x2, x3);
+      v[e] = __float_as_uint(x0);
+      v[e + 1] = __float_as_uint(x1);
+      v[e + 2] = __float_as_uint(x2);
+      v[e + 3] = __float_as_uint(x3);
+    }
+    const uint32_t row = sbuf + hr * C::HW;
+#pragma unroll
+    for (int u = 0; u < NU; ++u) {
+      const uint32_t w[4] = {v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]};
+      tmem_st4(row + (PB + u) * 4, w);
+    }
+  };
+  {
+    uint32_t va[NV], vb[NV];
+    load_pieces<C::HW, PB, NU>(sbuf + u_r0 * C::HW, va);
+    tmem_wait_ld();
+    for (int hr = u_r0; hr < u_r1; hr += 2) {
+      load_pieces<C::HW, PB, NU>(sbuf + min(hr + 1, u_r1 - 1) * C::HW, vb);
+      bias_row(hr, va);
+      tmem_wait_ld();
+      load_pieces<C::HW, PB, NU>(sbuf + min(hr + 2, u_r1 - 1) * C::HW, va);
+      if (hr + 1 < u_r1) bias_row(hr + 1, vb);
+      tmem_wait_ld();
+    }
+  }
+  tmem_wait_st();
+  const float mc = fmaxf(m0, m1) * c;
+
+  float l0 = 0.f, l1 = 0.f;
+  auto exp_row = [&](int hr, const uint32_t (&v)[NV]) {
+    uint32_t pk[C::HW / 2];
+#pragma unroll
+    for (int e = 0; e < C::HW / 2; ++e) pk[e] = 0u;
+#pragma unroll
+    for (int e = 0; e < NV; e += 4) {
+      float a0, a1, a2, a3;
+      fma2(a0, a1, __uint_as_float(v[e]), __uint_as_float(v[e + 1]), c, c, -mc, -mc);
+      fma2(a2, a3, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]), c, c, -mc, -mc);
+      const float p0 = ex2(a0), p1 = ex2(a1), p2 = ex2(a2), p3 = ex2(a3);
+      add2(l0, l1, l0, l1, p0, p1);
+      add2(l0, l1, l0, l1, p2, p3);
+      pk[PB * 2 + e / 2] = pack2<T>(p0, p1);
+      pk[PB * 2 + e / 2 + 1] = pack2<T>(p2, p3);
+    }
+    tmem_st_row(sbuf + hr * (C::HW / 2), pk);
+  };
+  {
+    uint32_t z[C::HW / 2];
+#pragma unroll
+    for (int e = 0; e < C::HW / 2; ++e) z[e] = 0u;
+    for (int hr = 0; hr < u_r0; ++hr) tmem_st_row(sbuf + hr * (C::HW / 2), z);
+  }
+  {
+    uint32_t va[NV], vb[NV];
+    load_pieces<C::HW, PB, NU>(sbuf + u_r0 * C::HW, va);
+    tmem_wait_ld();
+    for (int hr = u_r0; hr < u_r1; hr += 2) {
+      load_pieces<C::HW, PB, NU>(sbuf + min(hr + 1, u_r1 - 1) * C::HW, vb);
+      exp_row(hr, va);
+      tmem_wait_ld();
+      load_pieces<C::HW, PB, NU>(sbuf + min(hr + 2, u_r1 - 1) * C::HW, va);
+      if (hr + 1 < u_r1) exp_row(hr + 1, vb);
+      tmem_wait_ld();
+    }
+  }
+  {
+    uint32_t z[C::HW / 2];
+#pragma unroll
+    for (int e = 0; e < C::HW / 2; ++e) z[e] = 0u;
+    for (int hr = u_r1; hr < C::HH; ++hr) tmem_st_row(sbuf + hr * (C::HW / 2), z);
+  }
+  return l0 + l1;
+}
+
+// Runs softmax_rows with the pieces [pb, pb + NPU) fixed at compile time
+// (the common case), or over whole rows when the union is wider.
+template <typename T, int KS, int D, int PB = 0>
+NA_DEVICE float softmax_dispatch(int pb, int pe, uint32_t sbuf, const float* tbl, int u_r0, int u_r1, int wr0,
+                                 int er, int colbase, float c) {
+  using C = Cfg<KS, D>;
+  if constexpr (PB + C::NPU <= C::NPC) {
+    if (pe - pb <= C::NPU && min(pb, C::NPC - C::NPU) == PB)
+      return softmax_rows<T, KS, D, PB, C::NPU>(sbuf, tbl, u_r0, u_r1, wr0, er, colbase, c);
+    return softmax_dispatch<T, KS, D, PB + 1>(pb, pe, sbuf, tbl, u_r0, u_r1, wr0, er, colbase, c);
+  } else {
+    return softmax_rows<T, KS, D, 0, C::NPC>(sbuf, tbl, u_r0, u_r1, wr0, er, colbase, c);
+  }
+}
+
 template <typename T, int KS, int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<KS, D>::THREADS, 1)
 na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const Params p) {
   using C = Cfg<KS, D>;
   constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
+  constexpr int NB = C::NBUF, ST = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
-  float* tbl = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::TBL_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 3);
+  float* tables = reinterpret_cast<float*>(smem + ST * C::STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ST * C::STAGE_BYTES + NB * C::TBL_BYTES);
+  // barrier slots: full[ST] empty[ST] s_full[NB] p_full[NB] o_full[NB] o_empty[NB]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * ST + 4 * NB);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  auto bar_full = [&](int s) { return smem_addr(bars + s); };
-  auto bar_empty = [&](int s) { return smem_addr(bars + C::STAGES + s); };
-  const uint32_t bar_s_full = smem_addr(bars + 2 * C::STAGES);
-  const uint32_t bar_p_full = smem_addr(bars + 2 * C::STAGES + 1);
-  const uint32_t bar_o_full = smem_addr(bars + 2 * C::STAGES + 2);
+  auto bar = [&](int i) { return smem_addr(bars + i); };
+  auto bar_full = [&](int s) { return bar(s); };
+  auto bar_empty = [&](int s) { return bar(ST + s); };
+  auto bar_s_full = [&](int b) { return bar(2 * ST + b); };
+  auto bar_p_full = [&](int b) { return bar(2 * ST + NB + b); };
+  auto bar_o_full = [&](int b) { return bar(2 * ST + 2 * NB + b); };
+  auto bar_o_empty = [&](int b) { return bar(2 * ST + 3 * NB + b); };
   auto q_smem = [&](int s) { return sbase + s * C::STAGE_BYTES; };
   auto k_smem = [&](int s) { return sbase + s * C::STAGE_BYTES + C::Q_BYTES; };
   auto v_smem = [&](int s) { return sbase + s * C::STAGE_BYTES + C::Q_BYTES + C::KV_BYTES; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // The query operand of S = Q K^T is block structured: K block 0 holds
+  // tile A's queries (TMEM lanes 0-15 of every quarter), K block 1 tile B's
+  // (lanes 16-31); the other rows of each block stay zero.
+  for (int s = 0; s < ST; ++s)
+    for (int i = threadIdx.x; i < C::Q_BYTES / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(smem + s * C::STAGE_BYTES)[i] = make_uint4(0u, 0u, 0u, 0u);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
+    for (int s = 0; s < ST; ++s) {
       mbar_init(bar_full(s), 1);
       mbar_init(bar_empty(s), 1);
     }
-    mbar_init(bar_s_full, 1);
-    mbar_init(bar_p_full, 32 * kSoftmaxWarps);
-    mbar_init(bar_o_full, 1);
+    for (int b = 0; b < NB; ++b) {
+      mbar_init(bar_s_full(b), 1);
+      mbar_init(bar_p_full(b), 128);
+      mbar_init(bar_o_full(b), 1);
+      mbar_init(bar_o_empty(b), 128);
+    }
     *abort_flag = 0;
     mbar_init_fence();
     tma_prefetch_desc(&tm_q);
@@ -162,183 +338,170 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
       int n = 0;
-      for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++n) {
-        const int s = n % C::STAGES;
-        if (!mbar_wait(bar_empty(s), ((n / C::STAGES) & 1) ^ 1, abort_flag, p.status)) break;
-        const Tile tl = decode_tile<KS>(t, p);
-        mbar_expect_tx(bar_full(s), C::STAGE_BYTES);
-        for (int pq = 0; pq < 4; ++pq)
-          tma_load_5d(q_smem(s) + pq * PH * PW * C::ROWB, &tm_q, bar_full(s), 0, tl.j0 + (pq & 1) * PW,
-                      tl.i0 + (pq >> 1) * PH, tl.h, tl.b);
-        tma_load_5d(k_smem(s), &tm_k, bar_full(s), 0, tl.c0, tl.r0, tl.h, tl.b);
-        tma_load_5d(v_smem(s), &tm_v, bar_full(s), 0, tl.c0, tl.r0, tl.h, tl.b);
+      for (int t = blockIdx.x; t < p.total; t += gridDim.x, ++n) {
+        const int s = n % ST;
+        if (!mbar_wait(bar_empty(s), ((n / ST) & 1) ^ 1, abort_flag, p.status)) break;
+        const Pair pr = decode_pair<KS>(t, p);
+        mbar_expect_tx(bar_full(s), C::STAGE_BYTES - C::Q_BYTES / 2);
+#pragma unroll
+        for (int tile = 0; tile < 2; ++tile)
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            tma_load_5d(q_smem(s) + tile * C::QBLK + (32 * q + 16 * tile) * C::ROWB, &tm_q, bar_full(s), 0,
+                        pr.j0 + (q & 1) * PQ, pr.i0 + tile * TT + (q >> 1) * PQ, pr.h, pr.b);
+        tma_load_5d(k_smem(s), &tm_k, bar_full(s), 0, pr.c0, pr.R0, pr.h, pr.b);
+        tma_load_5d(v_smem(s), &tm_v, bar_full(s), 0, pr.c0, pr.R0, pr.h, pr.b);
       }
-      // drain: every stage's last use must have been released before exit
-      for (int e = 0; e < C::STAGES && !*abort_flag; ++e, ++n)
-        mbar_wait(bar_empty(n % C::STAGES), ((n / C::STAGES) & 1) ^ 1, abort_flag, p.status);
+      for (int e = 0; e < ST && !*abort_flag; ++e, ++n)
+        mbar_wait(bar_empty(n % ST), ((n / ST) & 1) ^ 1, abort_flag, p.status);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_pv = idesc_f16(kBF16, 128, D, true);
-      int n = 0;
-      for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++n) {
-        const int s = n % C::STAGES;
-        if (!mbar_wait(bar_full(s), (n / C::STAGES) & 1, abort_flag, p.status)) break;
-        tc_fence_after();
-        // S = Q . K_halo^T, in chunks of at most 256 keys
+      constexpr uint32_t idesc_pv = idesc_f16(kBF16, 128, 2 * D, true);
+      // Stages are contiguous, so a stage's descriptor is the first one plus
+      // s * STAGE_BYTES / 16 in the start-address field.
+      const uint64_t dq0 = smem_desc(q_smem(0), 16, 8 * C::ROWB, C::LAYOUT);
+      const uint64_t dk0 = smem_desc(k_smem(0), 16, 8 * C::ROWB, C::LAYOUT);
+      constexpr uint64_t kStageDesc = C::STAGE_BYTES >> 4;
+      auto issue_qk = [&](int n, const Pair& pr) {
+        const int s = n % ST, b = n % NB, use = n / NB;
+        // O of this buffer's previous pair overlays S: its epilogue must be done
+        if (!mbar_wait(bar_o_empty(b), (use & 1) ^ 1, abort_flag, p.status)) return false;
+        const uint32_t d = tmem + b * C::BUF_COLS;
+        const uint64_t qA = dq0 + s * kStageDesc, qB = qA + (C::QBLK >> 4);
+        const uint64_t kA = dk0 + s * kStageDesc, kB = kA + (uint64_t)(pr.rB * C::HW * C::ROWB >> 4);
 #pragma unroll
         for (int n0 = 0; n0 < C::NS; n0 += 256) {
           const int N = C::NS - n0 < 256 ? C::NS - n0 : 256;
           const uint32_t idesc = idesc_f16(kBF16, 128, N, false);
+          const uint64_t no = (uint64_t)(n0 * C::ROWB >> 4);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ad = smem_desc(q_smem(s) + kk * 32, 16, 8 * C::ROWB, C::LAYOUT);
-            const uint64_t bd = smem_desc(k_smem(s) + n0 * C::ROWB + kk * 32, 16, 8 * C::ROWB, C::LAYOUT);
-            mma_ss(tmem + C::S_COL + n0, ad, bd, idesc, kk > 0);
-          }
+          for (int kk = 0; kk < D / 16; ++kk) mma_ss(d + n0, qA + kk * 2, kA + no + kk * 2, idesc, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) mma_ss(d + n0, qB + kk * 2, kB + no + kk * 2, idesc, 1u);
         }
-        mma_commit(bar_s_full);
-        if (!mbar_wait(bar_p_full, n & 1, abort_flag, p.status)) break;
+        mma_commit(bar_s_full(b));
+        return true;
+      };
+      auto issue_pv = [&](int n, const Pair& pr) {
+        const int s = n % ST, b = n % NB, use = n / NB;
+        if (!mbar_wait(bar_p_full(b), use & 1, abort_flag, p.status)) return false;
         tc_fence_after();
-        // O = P . V_halo; P (16-bit, two keys per column) overlays S
-#pragma unroll 4
-        for (int kk = 0; kk < C::NS / 16; ++kk) {
-          const uint64_t bd = smem_desc(v_smem(s) + kk * 16 * C::ROWB, 16, 8 * C::ROWB, C::LAYOUT);
-          mma_ts(tmem + C::O_COL, tmem + C::S_COL + kk * 8, bd, idesc_pv, kk > 0);
-        }
-        mma_commit(bar_o_full);
+        const uint32_t a = tmem + b * C::BUF_COLS;
+        const uint32_t o = a + C::PO;
+        // B = [V_A | V_B]: two MN blocks of d columns, tile B's rows rB halo rows further on
+        const uint64_t vd = smem_desc(v_smem(s), (uint32_t)(pr.rB * C::HW * C::ROWB), 8 * C::ROWB, C::LAYOUT);
+        constexpr uint64_t kstep = 16 * C::ROWB >> 4;
+        mma_ts(o, a, vd, idesc_pv, 0u);
+#pragma unroll
+        for (int kk = 1; kk < C::NS / 16; ++kk) mma_ts(o, a + kk * 8, vd + kk * kstep, idesc_pv, 1u);
+        mma_commit(bar_o_full(b));
         mma_commit(bar_empty(s));
+        return true;
+      };
+      // P.V of pair n-1 goes before S of pair n when they share a tensor-memory
+      // buffer (NB == 1) or when pair n needs the shared-memory stage that only
+      // that P.V releases (ST == 1); otherwise after, so S of pair n overlaps
+      // the softmax of pair n-1.
+      constexpr bool kPvFirst = NB == 1 || ST == 1;
+      int n = 0;
+      Pair prev{};
+      for (int t = blockIdx.x; t < p.total; t += gridDim.x, ++n) {
+        const Pair pr = decode_pair<KS>(t, p);
+        if (kPvFirst && n > 0 && !issue_pv(n - 1, prev)) break;
+        if (!mbar_wait(bar_full(n % ST), (n / ST) & 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        if (!issue_qk(n, pr)) break;
+        if (!kPvFirst && n > 0 && !issue_pv(n - 1, prev)) break;
+        prev = pr;
       }
+      if (n > 0 && !*abort_flag) issue_pv(n - 1, prev);
     }
     __syncwarp();
   } else {
-    // ---------------------------------------------- softmax and epilogue
-    const int wq = warp & 3;  // tensor-memory lane quarter of this warp
-    const int pr0 = (wq >> 1) * PH, pc0 = (wq & 1) * PW;
-    const int qr = lane / PW, qc = lane % PW;
+    // ----------------------------------------- softmax groups + epilogue
+    const int g = (warp - 2) >> 2;  // group = tensor-memory buffer
+    const int wq = warp & 3;        // lane quarter
+    const int gtid = threadIdx.x - 64 - 128 * g;
+    const int tile = lane >> 4, l16 = lane & 15;
+    const int pr0 = (wq >> 1) * PQ + tile * TT + (l16 >> 2);  // query row inside the pair
+    const int pc0 = (wq & 1) * PQ + (l16 & 3);                // query column inside the pair
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
-    const int tid = threadIdx.x - 64;  // 0 .. 127
+    const uint32_t sbuf = tmem + lane_base + g * C::BUF_COLS;
+    float* tbl = tables + g * (C::TBL_BYTES / 4);
     const float c = p.scale_log2;
     const T* rpb = static_cast<const T*>(p.rpb);
     T* out = static_cast<T*>(p.out);
     int cur_h = -1;
-    int n = 0;
-    for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++n) {
-      const Tile tl = decode_tile<KS>(t, p);
-      if (tl.h != cur_h) {
-        // (re)build the bias / mask table of this head
-        named_barrier(1, 32 * kSoftmaxWarps);
+    int use = 0;
+    for (int t = blockIdx.x + g * gridDim.x; t < p.total; t += NB * gridDim.x, ++use) {
+      const Pair pr = decode_pair<KS>(t, p);
+      if (pr.h != cur_h) {
+        named_barrier(1 + g, 128);
         constexpr int span = 2 * KS - 1;
-        for (int idx = tid; idx < C::TBL_ROWS * C::TBL_W; idx += 32 * kSoftmaxWarps) {
+        for (int idx = gtid; idx < C::TBL_ROWS * C::TBL_W; idx += 128) {
           const int row = idx / C::TBL_W, col = idx % C::TBL_W;
           const int blk = col / (KS + C::PAD), off = col % (KS + C::PAD);
           float v = -INFINITY;
           if (row < span && blk < KS && off >= C::PAD) {
             const int bc = blk + (off - C::PAD);
-            v = rpb ? to_f(rpb[((size_t)tl.h * span + row) * span + bc]) : 0.f;
+            v = rpb ? to_f(rpb[((size_t)pr.h * span + row) * span + bc]) : 0.f;
           }
           tbl[idx] = v;
         }
-        named_barrier(1, 32 * kSoftmaxWarps);
-        cur_h = tl.h;
+        named_barrier(1 + g, 128);
+        cur_h = pr.h;
       }
-      const int i = tl.i0 + pr0 + qr, j = tl.j0 + pc0 + qc;
+      const int i = pr.i0 + pr0, j = pr.j0 + pc0;
       const bool valid = i < p.H && j < p.W;
       const int ic = min(i, p.H - 1), jc = min(j, p.W - 1);
       const int si = window_start(ic, p.H, KS), sj = window_start(jc, p.W, KS);
-      const int wr0 = si - tl.r0, wc0 = sj - tl.c0;         // window origin in the halo
-      const int er = tl.r0 - ic + KS - 1;                   // bias row of halo row 0
+      const int rt = pr.R0 + (tile ? pr.rB : 0);               // this tile's halo row origin
+      const int wr0 = si - rt, wc0 = sj - pr.c0;               // window origin in the tile halo
+      const int er = rt - ic + KS - 1;                         // bias row of halo row 0
       const int colbase = (sj - jc + KS - 1) * (KS + C::PAD) + C::PAD - wc0;
       const int u_r0 = __reduce_min_sync(0xffffffffu, wr0);
       const int u_r1 = __reduce_max_sync(0xffffffffu, wr0 + KS);
-      const int pbeg = __reduce_min_sync(0xffffffffu, wc0) >> 3;
-      const int pend = (__reduce_max_sync(0xffffffffu, wc0 + KS) + 7) >> 3;
+      const int pb = __reduce_min_sync(0xffffffffu, wc0) >> 2;
+      const int pe = (__reduce_max_sync(0xffffffffu, wc0 + KS) + 3) >> 2;
 
-      if (!mbar_wait(bar_s_full, n & 1, abort_flag, p.status)) break;
+      if (!mbar_wait(bar_s_full(g), use & 1, abort_flag, p.status)) break;
       tc_fence_after();
-      const uint32_t srow0 = tmem + lane_base + C::S_COL;
-
-      // pass 1: row maximum of the logits over the window
-      float m = -INFINITY;
-      for (int hr = u_r0; hr < u_r1; ++hr) {
-        uint32_t sv[C::NP][8];
-#pragma unroll
-        for (int pp = 0; pp < C::NP; ++pp)
-          if (pp >= pbeg && pp < pend) tmem_ld8(srow0 + hr * C::HW + pp * 8, sv[pp]);
-        tmem_wait_ld();
-        const float* trow = tbl + ((unsigned)(hr - wr0) < (unsigned)KS ? hr + er : 2 * KS - 1) * C::TBL_W + colbase;
-#pragma unroll
-        for (int pp = 0; pp < C::NP; ++pp)
-          if (pp >= pbeg && pp < pend) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) m = fmaxf(m, __uint_as_float(sv[pp][e]) + trow[pp * 8 + e]);
-          }
-      }
-      const float mc = m * c;
-
-      // pass 2: weights, row sum, P over S (every halo row, zeros outside the union)
-      float l = 0.f;
-      for (int hr = 0; hr < C::HH; ++hr) {
-        uint32_t pk[C::NP][4];
-        if (hr >= u_r0 && hr < u_r1) {
-          uint32_t sv[C::NP][8];
-#pragma unroll
-          for (int pp = 0; pp < C::NP; ++pp)
-            if (pp >= pbeg && pp < pend) tmem_ld8(srow0 + hr * C::HW + pp * 8, sv[pp]);
-          tmem_wait_ld();
-          const float* trow =
-              tbl + ((unsigned)(hr - wr0) < (unsigned)KS ? hr + er : 2 * KS - 1) * C::TBL_W + colbase;
-#pragma unroll
-          for (int pp = 0; pp < C::NP; ++pp) {
-            if (pp >= pbeg && pp < pend) {
-#pragma unroll
-              for (int e = 0; e < 8; e += 2) {
-                const float x0 = __uint_as_float(sv[pp][e]) + trow[pp * 8 + e];
-                const float x1 = __uint_as_float(sv[pp][e + 1]) + trow[pp * 8 + e + 1];
-                const float p0 = ex2(fmaf(x0, c, -mc));
-                const float p1 = ex2(fmaf(x1, c, -mc));
-                l += p0 + p1;
-                pk[pp][e >> 1] = pack2<T>(p0, p1);
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) pk[pp][e] = 0u;
-            }
-          }
-        } else {
-#pragma unroll
-          for (int pp = 0; pp < C::NP; ++pp)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) pk[pp][e] = 0u;
-        }
-        const uint32_t prow = srow0 + hr * (C::HW / 2);
-#pragma unroll
-        for (int pp = 0; pp < C::NP; ++pp) tmem_st4(prow + pp * 4, pk[pp]);
-      }
+      const float l = softmax_dispatch<T, KS, D>(pb, pe, sbuf, tbl, u_r0, u_r1, wr0, er, colbase, c);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_p_full);
+      mbar_arrive(bar_p_full(g));
 
-      // epilogue: O / l, rounded to T
-      if (!mbar_wait(bar_o_full, n & 1, abort_flag, p.status)) break;
+      // epilogue: O / l, rounded to T (tile A's columns, then tile B's)
+      if (!mbar_wait(bar_o_full(g), use & 1, abort_flag, p.status)) break;
       tc_fence_after();
-      uint32_t ov[D];
+      T* dst = out + ((((size_t)pr.b * p.heads + pr.h) * p.H + ic) * p.W + jc) * D;
+      const float inv = 1.f / l;
 #pragma unroll
-      for (int cc = 0; cc < D; cc += 32) tmem_ld32(tmem + lane_base + C::O_COL + cc, ov + cc);
-      tmem_wait_ld();
-      if (valid) {
-        const float inv = 1.f / l;
-        T* dst = out + ((((size_t)tl.b * p.heads + tl.h) * p.H + i) * p.W + j) * D;
+      for (int cc = 0; cc < D; cc += 32) {
+        uint32_t oa[32], ob[32];
+        tmem_ld32(sbuf + C::PO + cc, oa);
+        tmem_ld32(sbuf + C::PO + D + cc, ob);
+        tmem_wait_ld();
+        if (cc + 32 >= D) {
+          tc_fence_before();
+          mbar_arrive(bar_o_empty(g));
+        }
+        if (valid) {
 #pragma unroll
-        for (int x = 0; x < D; x += 8) {
-          uint4 w;
-          w.x = pack2<T>(__uint_as_float(ov[x + 0]) * inv, __uint_as_float(ov[x + 1]) * inv);
-          w.y = pack2<T>(__uint_as_float(ov[x + 2]) * inv, __uint_as_float(ov[x + 3]) * inv);
-          w.z = pack2<T>(__uint_as_float(ov[x + 4]) * inv, __uint_as_float(ov[x + 5]) * inv);
-          w.w = pack2<T>(__uint_as_float(ov[x + 6]) * inv, __uint_as_float(ov[x + 7]) * inv);
-          *reinterpret_cast<uint4*>(dst + x) = w;
+          for (int x = 0; x < 32; x += 8) {
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(tile ? ob[x + e] : oa[x + e]) * inv;
+            uint4 w;
+            w.x = pack2<T>(f[0], f[1]);
+            w.y = pack2<T>(f[2], f[3]);
+            w.z = pack2<T>(f[4], f[5]);
+            w.w = pack2<T>(f[6], f[7]);
+            *reinterpret_cast<uint4*>(dst + cc + x) = w;
+          }
         }
       }
     }
@@ -398,8 +561,8 @@ cudaError_t launch(const void* q, const void* k, const void* v, const void* rpb,
   using C = Cfg<KS, D>;
   constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, s, bf16, PW, PH) || !make_map(&mk, k, s, bf16, C::HW, C::HH) ||
-      !make_map(&mv, v, s, bf16, C::HW, C::HH))
+  if (!make_map(&mq, q, s, bf16, PQ, PQ) || !make_map(&mk, k, s, bf16, C::HW, C::HHP) ||
+      !make_map(&mv, v, s, bf16, C::HW, C::HHP))
     return cudaErrorInvalidValue;
   auto kern = na2d_fwd_tc_kernel<T, KS, D>;
   static std::mutex mu;
@@ -421,17 +584,17 @@ cudaError_t launch(const void* q, const void* k, const void* v, const void* rpb,
   p.heads = s.heads;
   p.H = s.H;
   p.W = s.W;
-  p.n_tr = (s.H + TH - 1) / TH;
-  p.n_tc = (s.W + TW - 1) / TW;
-  const long long tiles = (long long)p.n_tr * p.n_tc * s.B * s.heads;
-  if (tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
-  p.total_tiles = (int)tiles;
+  p.n_pr = (s.H + 2 * TT - 1) / (2 * TT);
+  p.n_pc = (s.W + TT - 1) / TT;
+  const long long pairs = (long long)p.n_pr * p.n_pc * s.B * s.heads;
+  if (pairs > 0x7fffffffLL) return cudaErrorInvalidValue;
+  p.total = (int)pairs;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)s.d));
   p.status = status;
   const int sms = sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
-  const int grid = p.total_tiles < sms ? p.total_tiles : sms;
-  kern<<<grid, kThreads, C::SMEM_BYTES, st>>>(mq, mk, mv, p);
+  const int grid = p.total < sms ? p.total : sms;
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, p);
   return cudaGetLastError();
 }
 
@@ -443,6 +606,10 @@ cudaError_t launch_ks(const void* q, const void* k, const void* v, const void* r
     case 5: return launch<T, 5, D>(q, k, v, rpb, out, s, status, st);
     case 7: return launch<T, 7, D>(q, k, v, rpb, out, s, status, st);
     case 9: return launch<T, 9, D>(q, k, v, rpb, out, s, status, st);
+    case 11: return launch<T, 11, D>(q, k, v, rpb, out, s, status, st);
+    case 13:
+      if constexpr (D == 32) return launch<T, 13, D>(q, k, v, rpb, out, s, status, st);
+      break;
   }
   return cudaErrorInvalidValue;
 }
@@ -452,7 +619,8 @@ cudaError_t launch_ks(const void* q, const void* k, const void* v, const void* r
 bool forward_tc_supported(const Shape& s, na_dtype dt) {
   if (dt != NA_F16 && dt != NA_BF16) return false;
   if (s.d != 32 && s.d != 64) return false;
-  if (s.ks != 3 && s.ks != 5 && s.ks != 7 && s.ks != 9) return false;
+  if (s.ks < 3 || s.ks > 13 || (s.ks & 1) == 0) return false;
+  if (s.ks == 13 && s.d != 32) return false;  // S + O would exceed tensor memory
   return true;
 }
 
