@@ -65,6 +65,13 @@ struct Cfg {
   static constexpr int NBUF = NS <= kTmemCols / 2 ? 2 : 1;
   static constexpr int BUF_COLS = kTmemCols / NBUF;
   static constexpr int PO = round_up(NS / 2, 32);
+  // When two S buffers and one O (2d columns) fit side by side, O is shared
+  // by the two buffers instead of overlaying S: S of a buffer's next pair
+  // can then be computed as soon as P.V has consumed P, before the epilogue.
+  static constexpr bool SHARED_O = NBUF == 2 && 2 * NS + 2 * D <= kTmemCols;
+  static constexpr int NO = SHARED_O ? 1 : NBUF;  // O buffers
+  static constexpr int s_col(int b) { return SHARED_O ? b * NS : b * BUF_COLS; }
+  static constexpr int o_col(int b) { return SHARED_O ? 2 * NS : b * BUF_COLS + PO; }
   // bias / mask table (one per softmax group): rows 0..2KS-2 hold bias rows,
   // row 2KS-1 is all -inf.  A row is KS blocks of stride KS+PAD; block dc
   // holds the bias row's columns dc..dc+KS-1 after PAD entries of -inf, and
@@ -75,14 +82,26 @@ struct Cfg {
   static constexpr int TBL_W = TBL_W0 + ((8 - TBL_W0 % 32) + 32) % 32;  // = 8 mod 32: conflict-free rows
   static constexpr int TBL_ROWS = 2 * KS;
   static constexpr int TBL_BYTES = TBL_ROWS * TBL_W * 4;
-  static constexpr int FIXED = 1024 + NBUF * TBL_BYTES + 512;
+  static constexpr int RAW = (2 * KS - 1) * (2 * KS - 1);  // one head's bias table
+  static constexpr int RAW_BYTES = round_up(RAW * 4, 16);
+  static constexpr int FIXED = 1024 + NBUF * (TBL_BYTES + RAW_BYTES) + 512;  // + barriers, TMEM slot
   static constexpr int STAGES_FIT = (kMaxSmem - FIXED) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT >= 3 ? 3 : STAGES_FIT;
   static constexpr int SMEM_RAW = FIXED + STAGES * STAGE_BYTES;
   static constexpr int SMEM_BYTES = SMEM_RAW > kMinSmem ? SMEM_RAW : kMinSmem;
-  static constexpr int THREADS = 64 + 128 * NBUF;
+  // warpgroup 0: TMA producer (warp 0), MMA issuer (warp 1), two idle warps;
+  // warpgroups 1..NBUF: softmax groups.  With two softmax groups the register
+  // file is re-split at run time: the control warpgroup keeps REGS_CTRL per
+  // thread, the softmax groups grow to REGS_SOFTMAX, which together use
+  // exactly the registers a 384-thread CTA is launched with (168 each).
+  static constexpr int THREADS = 128 * (1 + NBUF);
+  static constexpr int LAUNCH_REGS = 168;
+  static constexpr int REGS_CTRL = KS <= 5 ? 80 : 72, REGS_SOFTMAX = KS <= 5 ? 208 : 216;
+  static_assert(NBUF == 1 || REGS_CTRL * 128 + REGS_SOFTMAX * 256 <= LAUNCH_REGS * THREADS,
+                "the register split must fit the launch allocation");
   static constexpr uint32_t LAYOUT = ROWB == 64 ? kLayoutSW64 : kLayoutSW128;
   static_assert(NS <= BUF_COLS && PO + 2 * D <= BUF_COLS, "S, P and O of a buffer must fit in tensor memory");
+  static_assert(!SHARED_O || NS % 32 == 0, "buffers start on 32-column boundaries");
   static_assert(STAGES >= 1, "a pipeline stage must fit in shared memory");
   static_assert(NS % 16 == 0, "halo keys must be a multiple of the MMA K step");
   static_assert(QBLK % 1024 == 0 && KV_BYTES % 1024 == 0 && (TT * HW * ROWB) % 1024 == 0,
@@ -105,22 +124,52 @@ struct Pair {
   int b, h, i0, j0, R0, c0, rB;
 };
 
-template <int KS>
-NA_DEVICE Pair decode_pair(int t, const Params& p) {
-  Pair q;
-  const int pc = t % p.n_pc;
-  int rest = t / p.n_pc;
-  const int pr = rest % p.n_pr;
-  rest /= p.n_pr;
-  q.b = rest % p.B;
-  q.h = rest / p.B;
-  q.i0 = pr * 2 * TT;
-  q.j0 = pc * TT;
-  q.R0 = window_start(q.i0, p.H, KS);
-  q.rB = window_start(min(q.i0 + TT, p.H - 1), p.H, KS) - q.R0;  // 0 .. 8
-  q.c0 = min(q.j0 - KS / 2, window_start(q.j0, p.W, KS));
-  return q;
-}
+// Walks the pair indices t, t + stride, ... of one role.  Pair index order
+// is (head, batch, pair row, pair column), column fastest; the walk keeps
+// the four digits and adds the stride's digits with carries, so the loop
+// does no division.
+struct PairIter {
+  int t, pc, pr, b, h;            // current pair
+  int s0, s1, s2, s3, stride;     // the stride's digits
+  NA_DEVICE void digits(int x, const Params& p, int& d0, int& d1, int& d2, int& d3) {
+    d0 = x % p.n_pc;
+    x /= p.n_pc;
+    d1 = x % p.n_pr;
+    x /= p.n_pr;
+    d2 = x % p.B;
+    d3 = x / p.B;
+  }
+  NA_DEVICE PairIter(int t0, int stride_, const Params& p) : t(t0), stride(stride_) {
+    digits(t0, p, pc, pr, b, h);
+    digits(stride_, p, s0, s1, s2, s3);
+  }
+  NA_DEVICE bool valid(const Params& p) const { return t < p.total; }
+  NA_DEVICE void next(const Params& p) {
+    t += stride;
+    pc += s0;
+    int c = pc >= p.n_pc;
+    pc -= c ? p.n_pc : 0;
+    pr += s1 + c;
+    c = pr >= p.n_pr;
+    pr -= c ? p.n_pr : 0;
+    b += s2 + c;
+    c = b >= p.B;
+    b -= c ? p.B : 0;
+    h += s3 + c;
+  }
+  template <int KS>
+  NA_DEVICE Pair pair(const Params& p) const {
+    Pair q;
+    q.b = b;
+    q.h = h;
+    q.i0 = pr * 2 * TT;
+    q.j0 = pc * TT;
+    q.R0 = window_start(q.i0, p.H, KS);
+    q.rB = window_start(min(q.i0 + TT, p.H - 1), p.H, KS) - q.R0;  // 0 .. 8
+    q.c0 = min(q.j0 - KS / 2, window_start(q.j0, p.W, KS));
+    return q;
+  }
+};
 
 template <typename T> NA_DEVICE float to_f(T x);
 template <> NA_DEVICE float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -147,123 +196,142 @@ NA_DEVICE void tmem_st_row(uint32_t taddr, const uint32_t (&r)[N]) {
   }
 }
 
-// Loads pieces [PB, PB+NU) (4 columns each) of halo row `row` of S.
-template <int HW, int PB, int NU>
-NA_DEVICE void load_pieces(uint32_t row, uint32_t (&v)[NU * 4]) {
-  if constexpr (PB == 0 && NU * 4 == 16) {
-    tmem_ld16(row, v);
-  } else {
+// Largest access width (4, 8 or 16 columns) that a start column known to be
+// a multiple of `align` allows; every tensor-memory access starts at a
+// multiple of its own width.
+__host__ __device__ constexpr int span_width(int align) { return align % 16 == 0 ? 16 : align % 8 == 0 ? 8 : 4; }
+__host__ __device__ constexpr int low_pow2(int x) { return x & -x; }
+
+// N consecutive 32-bit columns starting at a column that is a multiple of A.
+template <int N, int A>
+NA_DEVICE void ld_span(uint32_t addr, uint32_t* v) {
+  static_assert(N % 4 == 0 && A % 4 == 0, "spans go by 4 columns");
+  constexpr int W = span_width(A) < span_width(N) ? span_width(A) : span_width(N);  // divides N and A
 #pragma unroll
-    for (int u = 0; u < NU; ++u) {
-      uint32_t w[4];
-      tmem_ld4(row + (PB + u) * 4, w);
+  for (int c = 0; c < N; c += W) {
+    if constexpr (W == 16) tmem_ld16(addr + c, *reinterpret_cast<uint32_t(*)[16]>(v + c));
+    else if constexpr (W == 8) tmem_ld8(addr + c, *reinterpret_cast<uint32_t(*)[8]>(v + c));
+    else tmem_ld4(addr + c, *reinterpret_cast<uint32_t(*)[4]>(v + c));
+  }
+}
+template <int N, int A>
+NA_DEVICE void st_span(uint32_t addr, const uint32_t* v) {
+  static_assert(N % 4 == 0 && A % 4 == 0, "spans go by 4 columns");
+  constexpr int W = span_width(A) < span_width(N) ? span_width(A) : span_width(N);  // divides N and A
 #pragma unroll
-      for (int e = 0; e < 4; ++e) v[4 * u + e] = w[e];
-    }
+  for (int c = 0; c < N; c += W) {
+    if constexpr (W == 16) tmem_st16(addr + c, v + c);
+    else if constexpr (W == 8) tmem_st8(addr + c, v + c);
+    else tmem_st4(addr + c, *reinterpret_cast<const uint32_t(*)[4]>(v + c));
   }
 }
 
-// Softmax of one warp's 32 queries (two 4x4 patches) over the union rows
-// [u_r0, u_r1) and pieces [PB, PB+NU) of their windows.  Pass 1 writes
-// x = s + bias (-inf outside the window) back over S and takes the row
-// maximum; pass 2 writes P = exp2(x c - max c) as 16-bit pairs over S (P
-// row hr covers the S columns of row hr/2, which pass 2 has already read)
-// and returns the row sum.  Rows are processed two at a time with the next
-// row's loads in flight.
+// exp2 of a float pair, rounded to T: two results per MUFU operation.  The
+// exponent argument is rounded to T first; for bf16 that adds at most about
+// 0.3% relative error to each weight, inside the bf16 rounding of P itself.
+template <typename T> NA_DEVICE uint32_t exp2_pair(float a0, float a1);
+template <> NA_DEVICE uint32_t exp2_pair<__nv_bfloat16>(float a0, float a1) {
+  return ex2_bf16x2(pack2<__nv_bfloat16>(a0, a1));
+}
+template <> NA_DEVICE uint32_t exp2_pair<__half>(float a0, float a1) { return ex2_f16x2(pack2<__half>(a0, a1)); }
+template <typename T> NA_DEVICE float2 unpack2(uint32_t w);
+template <> NA_DEVICE float2 unpack2<__nv_bfloat16>(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+template <> NA_DEVICE float2 unpack2<__half>(uint32_t w) { return __half22float2(*reinterpret_cast<__half2*>(&w)); }
+
+// Softmax of one warp's 32 queries (two 4x4 patches, one per tile) over the
+// union rows [u_r0, u_r1) and pieces [PB, PB+NU) of their windows, RB rows
+// at a time: each batch's tensor-memory loads are issued together and the RB
+// rows are independent streams of arithmetic.  Pass 1 writes
+// y = s log2e/sqrt(d) + table (bias log2e/sqrt(d), -inf outside the window)
+// back over S and takes the row maximum m; pass 2 writes P = exp2(y - m) as
+// 16-bit pairs over S -- P row hr covers the S columns of row hr / 2, read by
+// an earlier or the same batch -- zeros outside the pieces, and returns the
+// sum of the rounded P.  Rows past u_r1 in the last batch repeat row u_r1-1:
+// they store the same values again and are left out of the sum.
 template <typename T, int KS, int D, int PB, int NU>
-NA_DEVICE float softmax_rows(uint32_t sbuf, const float* tbl, int u_r0, int u_r1, int wr0, int er,
-                             int colbase, float c) {
+NA_DEVICE float softmax_rows(uint32_t sbuf, const float* tbl, int u_r0, int u_r1, int wr0, int er, int colbase,
+                             float c) {
   using C = Cfg<KS, D>;
-  constexpr int NV = NU * 4;
-  auto trow_of = [&](int hr) {
-    return tbl + ((unsigned)(hr - wr0) < (unsigned)KS ? hr + er : 2 * KS - 1) * C::TBL_W + colbase + PB * 4;
-  };
-  float m0 = -INFINITY, m1 = -INFINITY;
-  auto bias_row = [&](int hr, uint32_t (&v)[NV]) {
-    const float* tr = trow_of(hr);
+  constexpr int HW = C::HW, PW = HW / 2, NV = NU * 4, RB = 2;
+  // start-column alignment of a piece window (row hr * HW + PB * 4) and of a P row (hr * PW)
+  constexpr int AS = PB == 0 ? low_pow2(HW) : (low_pow2(HW) < low_pow2(PB * 4) ? low_pow2(HW) : low_pow2(PB * 4));
+  constexpr int AP = low_pow2(PW);
+  const int last = u_r1 - 1;
+  float mx[RB];
 #pragma unroll
-    for (int e = 0; e < NV; e += 4) {
-      float x0, x1, x2, x3;
-      add2(x0, x1, __uint_as_float(v[e]), __uint_as_float(v[e + 1]), tr[e], tr[e + 1]);
-      add2(x2, x3, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]), tr[e + 2], tr[e + 3]);
-      m0 = max3(m0, x0, x1);
-      m1 = max3(m1, x2, x3);
-      v[e] = __float_as_uint(x0);
-      v[e + 1] = __float_as_uint(x1);
-      v[e + 2] = __float_as_uint(x2);
-      v[e + 3] = __float_as_uint(x3);
-    }
-    const uint32_t row = sbuf + hr * C::HW;
+  for (int j = 0; j < RB; ++j) mx[j] = -INFINITY;
+  for (int r0 = u_r0; r0 < u_r1; r0 += RB) {
+    uint32_t v[RB][NV];
 #pragma unroll
-    for (int u = 0; u < NU; ++u) {
-      const uint32_t w[4] = {v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]};
-      tmem_st4(row + (PB + u) * 4, w);
-    }
-  };
-  {
-    uint32_t va[NV], vb[NV];
-    load_pieces<C::HW, PB, NU>(sbuf + u_r0 * C::HW, va);
-    tmem_wait_ld();
-    for (int hr = u_r0; hr < u_r1; hr += 2) {
-      load_pieces<C::HW, PB, NU>(sbuf + min(hr + 1, u_r1 - 1) * C::HW, vb);
-      bias_row(hr, va);
-      tmem_wait_ld();
-      load_pieces<C::HW, PB, NU>(sbuf + min(hr + 2, u_r1 - 1) * C::HW, va);
-      if (hr + 1 < u_r1) bias_row(hr + 1, vb);
-      tmem_wait_ld();
+    for (int j = 0; j < RB; ++j) ld_span<NV, AS>(sbuf + min(r0 + j, last) * HW + PB * 4, v[j]);
+#pragma unroll
+    for (int j = 0; j < RB; ++j) tmem_wait_ld_regs(v[j]);
+#pragma unroll
+    for (int j = 0; j < RB; ++j) {
+      const int hr = min(r0 + j, last);
+      const float* tr =
+          tbl + ((unsigned)(hr - wr0) < (unsigned)KS ? hr + er : 2 * KS - 1) * C::TBL_W + colbase + PB * 4;
+#pragma unroll
+      for (int e = 0; e < NV; e += 4) {
+        float y0, y1, y2, y3;
+        fma2(y0, y1, __uint_as_float(v[j][e]), __uint_as_float(v[j][e + 1]), c, c, tr[e], tr[e + 1]);
+        fma2(y2, y3, __uint_as_float(v[j][e + 2]), __uint_as_float(v[j][e + 3]), c, c, tr[e + 2], tr[e + 3]);
+        mx[j] = max3(mx[j], max3(y0, y1, y2), y3);
+        v[j][e] = __float_as_uint(y0);
+        v[j][e + 1] = __float_as_uint(y1);
+        v[j][e + 2] = __float_as_uint(y2);
+        v[j][e + 3] = __float_as_uint(y3);
+      }
+      st_span<NV, AS>(sbuf + hr * HW + PB * 4, v[j]);
     }
   }
   tmem_wait_st();
-  const float mc = fmaxf(m0, m1) * c;
+  float m = mx[0];
+#pragma unroll
+  for (int j = 1; j < RB; ++j) m = fmaxf(m, mx[j]);
 
-  float l0 = 0.f, l1 = 0.f;
-  auto exp_row = [&](int hr, const uint32_t (&v)[NV]) {
-    uint32_t pk[C::HW / 2];
+  uint32_t z[PW];
 #pragma unroll
-    for (int e = 0; e < C::HW / 2; ++e) pk[e] = 0u;
+  for (int e = 0; e < PW; ++e) z[e] = 0u;
+  for (int hr = 0; hr < u_r0; ++hr) st_span<PW, AP>(sbuf + hr * PW, z);
+  float l = 0.f;
+  for (int r0 = u_r0; r0 < u_r1; r0 += RB) {
+    uint32_t v[RB][NV];
 #pragma unroll
-    for (int e = 0; e < NV; e += 4) {
-      float a0, a1, a2, a3;
-      fma2(a0, a1, __uint_as_float(v[e]), __uint_as_float(v[e + 1]), c, c, -mc, -mc);
-      fma2(a2, a3, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]), c, c, -mc, -mc);
-      const float p0 = ex2(a0), p1 = ex2(a1), p2 = ex2(a2), p3 = ex2(a3);
-      add2(l0, l1, l0, l1, p0, p1);
-      add2(l0, l1, l0, l1, p2, p3);
-      pk[PB * 2 + e / 2] = pack2<T>(p0, p1);
-      pk[PB * 2 + e / 2 + 1] = pack2<T>(p2, p3);
-    }
-    tmem_st_row(sbuf + hr * (C::HW / 2), pk);
-  };
-  {
-    uint32_t z[C::HW / 2];
+    for (int j = 0; j < RB; ++j) ld_span<NV, AS>(sbuf + min(r0 + j, last) * HW + PB * 4, v[j]);
 #pragma unroll
-    for (int e = 0; e < C::HW / 2; ++e) z[e] = 0u;
-    for (int hr = 0; hr < u_r0; ++hr) tmem_st_row(sbuf + hr * (C::HW / 2), z);
-  }
-  {
-    uint32_t va[NV], vb[NV];
-    load_pieces<C::HW, PB, NU>(sbuf + u_r0 * C::HW, va);
-    tmem_wait_ld();
-    for (int hr = u_r0; hr < u_r1; hr += 2) {
-      load_pieces<C::HW, PB, NU>(sbuf + min(hr + 1, u_r1 - 1) * C::HW, vb);
-      exp_row(hr, va);
-      tmem_wait_ld();
-      load_pieces<C::HW, PB, NU>(sbuf + min(hr + 2, u_r1 - 1) * C::HW, va);
-      if (hr + 1 < u_r1) exp_row(hr + 1, vb);
-      tmem_wait_ld();
+    for (int j = 0; j < RB; ++j) tmem_wait_ld_regs(v[j]);
+#pragma unroll
+    for (int j = 0; j < RB; ++j) {
+      uint32_t pk[PW];
+#pragma unroll
+      for (int e = 0; e < PW; ++e) pk[e] = 0u;
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int e = 0; e < NV; e += 4) {
+        float a0, a1, a2, a3;
+        add2(a0, a1, __uint_as_float(v[j][e]), __uint_as_float(v[j][e + 1]), -m, -m);
+        add2(a2, a3, __uint_as_float(v[j][e + 2]), __uint_as_float(v[j][e + 3]), -m, -m);
+        const uint32_t pa = exp2_pair<T>(a0, a1), pb = exp2_pair<T>(a2, a3);
+        const float2 fa = unpack2<T>(pa), fb = unpack2<T>(pb);
+        add2(s0, s1, s0, s1, fa.x, fa.y);
+        add2(s0, s1, s0, s1, fb.x, fb.y);
+        pk[PB * 2 + e / 2] = pa;
+        pk[PB * 2 + e / 2 + 1] = pb;
+      }
+      st_span<PW, AP>(sbuf + min(r0 + j, last) * PW, pk);
+      if (r0 + j < u_r1) l += s0 + s1;
     }
   }
-  {
-    uint32_t z[C::HW / 2];
-#pragma unroll
-    for (int e = 0; e < C::HW / 2; ++e) z[e] = 0u;
-    for (int hr = u_r1; hr < C::HH; ++hr) tmem_st_row(sbuf + hr * (C::HW / 2), z);
-  }
-  return l0 + l1;
+  for (int hr = u_r1; hr < C::HH; ++hr) st_span<PW, AP>(sbuf + hr * PW, z);
+  return l;
 }
 
-// Runs softmax_rows with the pieces [pb, pb + NPU) fixed at compile time
-// (the common case), or over whole rows when the union is wider.
+// Runs softmax_rows over the pieces [pb, pb + NPU) of an interior patch's
+// window union, fixed at compile time, or over whole rows when the union is
+// wider (patches at the map border).
 template <typename T, int KS, int D, int PB = 0>
 NA_DEVICE float softmax_dispatch(int pb, int pe, uint32_t sbuf, const float* tbl, int u_r0, int u_r1, int wr0,
                                  int er, int colbase, float c) {
@@ -288,17 +356,26 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
   float* tables = reinterpret_cast<float*>(smem + ST * C::STAGE_BYTES);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ST * C::STAGE_BYTES + NB * C::TBL_BYTES);
-  // barrier slots: full[ST] empty[ST] s_full[NB] p_full[NB] o_full[NB] o_empty[NB]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * ST + 4 * NB);
+  float* raws = reinterpret_cast<float*>(smem + ST * C::STAGE_BYTES + NB * C::TBL_BYTES);
+  uint64_t* bars =
+      reinterpret_cast<uint64_t*>(smem + ST * C::STAGE_BYTES + NB * (C::TBL_BYTES + C::RAW_BYTES));
+  // barrier slots: full[ST][NB] empty[ST] s_full[NB] p_full[NB] o_full[NB] s_free[NB] o_empty[NO].
+  // A stage's "full" barrier is split by buffer: each is waited on by one
+  // issuer only, one phase per use, so a parity wait can never see a phase
+  // of a pair that belongs to the other buffer.  Pair n uses full[n % ST][n % NB],
+  // for the (n / LCM)-th time.
+  constexpr int LCM = (ST % NB == 0) ? ST : ST * NB;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + ST * NB + ST + 5 * NB);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto bar = [&](int i) { return smem_addr(bars + i); };
-  auto bar_full = [&](int s) { return bar(s); };
-  auto bar_empty = [&](int s) { return bar(ST + s); };
-  auto bar_s_full = [&](int b) { return bar(2 * ST + b); };
-  auto bar_p_full = [&](int b) { return bar(2 * ST + NB + b); };
-  auto bar_o_full = [&](int b) { return bar(2 * ST + 2 * NB + b); };
-  auto bar_o_empty = [&](int b) { return bar(2 * ST + 3 * NB + b); };
+  auto bar_full = [&](int n) { return bar((n % ST) * NB + n % NB); };
+  auto bar_empty = [&](int s) { return bar(ST * NB + s); };
+  constexpr int B0 = ST * NB + ST;
+  auto bar_s_full = [&](int b) { return bar(B0 + b); };
+  auto bar_p_full = [&](int b) { return bar(B0 + NB + b); };
+  auto bar_o_full = [&](int b) { return bar(B0 + 2 * NB + b); };
+  auto bar_s_free = [&](int b) { return bar(B0 + 3 * NB + b); };
+  auto bar_o_empty = [&](int o) { return bar(B0 + 4 * NB + o); };
   auto q_smem = [&](int s) { return sbase + s * C::STAGE_BYTES; };
   auto k_smem = [&](int s) { return sbase + s * C::STAGE_BYTES + C::Q_BYTES; };
   auto v_smem = [&](int s) { return sbase + s * C::STAGE_BYTES + C::Q_BYTES + C::KV_BYTES; };
@@ -312,16 +389,15 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       reinterpret_cast<uint4*>(smem + s * C::STAGE_BYTES)[i] = make_uint4(0u, 0u, 0u, 0u);
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   if (threadIdx.x == 0) {
-    for (int s = 0; s < ST; ++s) {
-      mbar_init(bar_full(s), 1);
-      mbar_init(bar_empty(s), 1);
-    }
+    for (int i = 0; i < ST * NB; ++i) mbar_init(bar(i), 1);
+    for (int s = 0; s < ST; ++s) mbar_init(bar_empty(s), 1);
     for (int b = 0; b < NB; ++b) {
       mbar_init(bar_s_full(b), 1);
       mbar_init(bar_p_full(b), 128);
       mbar_init(bar_o_full(b), 1);
-      mbar_init(bar_o_empty(b), 128);
+      mbar_init(bar_s_free(b), 1);
     }
+    for (int o = 0; o < C::NO; ++o) mbar_init(bar_o_empty(o), 128);
     *abort_flag = 0;
     mbar_init_fence();
     tma_prefetch_desc(&tm_q);
@@ -334,30 +410,37 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp < 4) {
+  if constexpr (NB == 2) regs_dec<C::REGS_CTRL>();
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
       int n = 0;
-      for (int t = blockIdx.x; t < p.total; t += gridDim.x, ++n) {
+      for (PairIter it(blockIdx.x, gridDim.x, p); it.valid(p); it.next(p), ++n) {
         const int s = n % ST;
         if (!mbar_wait(bar_empty(s), ((n / ST) & 1) ^ 1, abort_flag, p.status)) break;
-        const Pair pr = decode_pair<KS>(t, p);
-        mbar_expect_tx(bar_full(s), C::STAGE_BYTES - C::Q_BYTES / 2);
+        const Pair pr = it.pair<KS>(p);
+        const uint32_t full = bar_full(n);
+        mbar_expect_tx(full, C::STAGE_BYTES - C::Q_BYTES / 2);
 #pragma unroll
         for (int tile = 0; tile < 2; ++tile)
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            tma_load_5d(q_smem(s) + tile * C::QBLK + (32 * q + 16 * tile) * C::ROWB, &tm_q, bar_full(s), 0,
+            tma_load_5d(q_smem(s) + tile * C::QBLK + (32 * q + 16 * tile) * C::ROWB, &tm_q, full, 0,
                         pr.j0 + (q & 1) * PQ, pr.i0 + tile * TT + (q >> 1) * PQ, pr.h, pr.b);
-        tma_load_5d(k_smem(s), &tm_k, bar_full(s), 0, pr.c0, pr.R0, pr.h, pr.b);
-        tma_load_5d(v_smem(s), &tm_v, bar_full(s), 0, pr.c0, pr.R0, pr.h, pr.b);
+        tma_load_5d(k_smem(s), &tm_k, full, 0, pr.c0, pr.R0, pr.h, pr.b);
+        tma_load_5d(v_smem(s), &tm_v, full, 0, pr.c0, pr.R0, pr.h, pr.b);
       }
       for (int e = 0; e < ST && !*abort_flag; ++e, ++n)
         mbar_wait(bar_empty(n % ST), ((n / ST) & 1) ^ 1, abort_flag, p.status);
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------- MMA issuer
+  } else if (warp <= NB) {
+    // -------------------------------------------- MMA issuer of buffer b
+    // Buffer b takes the CTA's pairs b, b + NB, ...; its issuer runs
+    // S = Q K^T, then (after the softmax) O = P V, in that order, so the
+    // two buffers never wait on each other's barriers.
+    const int b = warp - 1;
     if (lane == 0) {
       constexpr uint32_t idesc_pv = idesc_f16(kBF16, 128, 2 * D, true);
       // Stages are contiguous, so a stage's descriptor is the first one plus
@@ -365,11 +448,20 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const uint64_t dq0 = smem_desc(q_smem(0), 16, 8 * C::ROWB, C::LAYOUT);
       const uint64_t dk0 = smem_desc(k_smem(0), 16, 8 * C::ROWB, C::LAYOUT);
       constexpr uint64_t kStageDesc = C::STAGE_BYTES >> 4;
-      auto issue_qk = [&](int n, const Pair& pr) {
-        const int s = n % ST, b = n % NB, use = n / NB;
-        // O of this buffer's previous pair overlays S: its epilogue must be done
-        if (!mbar_wait(bar_o_empty(b), (use & 1) ^ 1, abort_flag, p.status)) return false;
-        const uint32_t d = tmem + b * C::BUF_COLS;
+      const uint32_t d = tmem + C::s_col(b), o = tmem + C::o_col(b);
+      int n = b, use = 0;
+      for (PairIter it(blockIdx.x + b * gridDim.x, NB * gridDim.x, p); it.valid(p); it.next(p), n += NB, ++use) {
+        const Pair pr = it.pair<KS>(p);
+        const int s = n % ST;
+        if (!mbar_wait(bar_full(n), (n / LCM) & 1, abort_flag, p.status)) break;
+        // S of this buffer is free once the buffer's previous P.V has read P
+        // and, when O overlays S, once that pair's epilogue has read O.
+        if constexpr (C::SHARED_O) {
+          if (!mbar_wait(bar_s_free(b), (use & 1) ^ 1, abort_flag, p.status)) break;
+        } else {
+          if (!mbar_wait(bar_o_empty(b), (use & 1) ^ 1, abort_flag, p.status)) break;
+        }
+        tc_fence_after();
         const uint64_t qA = dq0 + s * kStageDesc, qB = qA + (C::QBLK >> 4);
         const uint64_t kA = dk0 + s * kStageDesc, kB = kA + (uint64_t)(pr.rB * C::HW * C::ROWB >> 4);
 #pragma unroll
@@ -383,72 +475,65 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           for (int kk = 0; kk < D / 16; ++kk) mma_ss(d + n0, qB + kk * 2, kB + no + kk * 2, idesc, 1u);
         }
         mma_commit(bar_s_full(b));
-        return true;
-      };
-      auto issue_pv = [&](int n, const Pair& pr) {
-        const int s = n % ST, b = n % NB, use = n / NB;
-        if (!mbar_wait(bar_p_full(b), use & 1, abort_flag, p.status)) return false;
+
+        if (!mbar_wait(bar_p_full(b), use & 1, abort_flag, p.status)) break;
+        // a shared O must have been read by the epilogue of the CTA's previous pair
+        if (C::SHARED_O && !mbar_wait(bar_o_empty(0), (n & 1) ^ 1, abort_flag, p.status)) break;
         tc_fence_after();
-        const uint32_t a = tmem + b * C::BUF_COLS;
-        const uint32_t o = a + C::PO;
         // B = [V_A | V_B]: two MN blocks of d columns, tile B's rows rB halo rows further on
         const uint64_t vd = smem_desc(v_smem(s), (uint32_t)(pr.rB * C::HW * C::ROWB), 8 * C::ROWB, C::LAYOUT);
         constexpr uint64_t kstep = 16 * C::ROWB >> 4;
-        mma_ts(o, a, vd, idesc_pv, 0u);
+        mma_ts(o, d, vd, idesc_pv, 0u);
 #pragma unroll
-        for (int kk = 1; kk < C::NS / 16; ++kk) mma_ts(o, a + kk * 8, vd + kk * kstep, idesc_pv, 1u);
+        for (int kk = 1; kk < C::NS / 16; ++kk) mma_ts(o, d + kk * 8, vd + kk * kstep, idesc_pv, 1u);
         mma_commit(bar_o_full(b));
         mma_commit(bar_empty(s));
-        return true;
-      };
-      // P.V of pair n-1 goes before S of pair n when they share a tensor-memory
-      // buffer (NB == 1) or when pair n needs the shared-memory stage that only
-      // that P.V releases (ST == 1); otherwise after, so S of pair n overlaps
-      // the softmax of pair n-1.
-      constexpr bool kPvFirst = NB == 1 || ST == 1;
-      int n = 0;
-      Pair prev{};
-      for (int t = blockIdx.x; t < p.total; t += gridDim.x, ++n) {
-        const Pair pr = decode_pair<KS>(t, p);
-        if (kPvFirst && n > 0 && !issue_pv(n - 1, prev)) break;
-        if (!mbar_wait(bar_full(n % ST), (n / ST) & 1, abort_flag, p.status)) break;
-        tc_fence_after();
-        if (!issue_qk(n, pr)) break;
-        if (!kPvFirst && n > 0 && !issue_pv(n - 1, prev)) break;
-        prev = pr;
+        if constexpr (C::SHARED_O) mma_commit(bar_s_free(b));
       }
-      if (n > 0 && !*abort_flag) issue_pv(n - 1, prev);
     }
     __syncwarp();
+  }
   } else {
+    if constexpr (NB == 2) regs_inc<C::REGS_SOFTMAX>();
     // ----------------------------------------- softmax groups + epilogue
-    const int g = (warp - 2) >> 2;  // group = tensor-memory buffer
+    const int g = (warp - 4) >> 2;  // group = tensor-memory buffer
     const int wq = warp & 3;        // lane quarter
-    const int gtid = threadIdx.x - 64 - 128 * g;
+    const int gtid = threadIdx.x - 128 - 128 * g;
     const int tile = lane >> 4, l16 = lane & 15;
     const int pr0 = (wq >> 1) * PQ + tile * TT + (l16 >> 2);  // query row inside the pair
     const int pc0 = (wq & 1) * PQ + (l16 & 3);                // query column inside the pair
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
-    const uint32_t sbuf = tmem + lane_base + g * C::BUF_COLS;
+    const uint32_t sbuf = tmem + lane_base + C::s_col(g);
+    const uint32_t obuf = tmem + lane_base + C::o_col(g);
     float* tbl = tables + g * (C::TBL_BYTES / 4);
+    float* raw = raws + g * (C::RAW_BYTES / 4);
     const float c = p.scale_log2;
     const T* rpb = static_cast<const T*>(p.rpb);
     T* out = static_cast<T*>(p.out);
     int cur_h = -1;
     int use = 0;
-    for (int t = blockIdx.x + g * gridDim.x; t < p.total; t += NB * gridDim.x, ++use) {
-      const Pair pr = decode_pair<KS>(t, p);
+    for (PairIter it(blockIdx.x + g * gridDim.x, NB * gridDim.x, p); it.valid(p); it.next(p), ++use) {
+      const Pair pr = it.pair<KS>(p);
       if (pr.h != cur_h) {
-        named_barrier(1 + g, 128);
+        // New head: stage its bias (times log2e / sqrt(d)) with all loads in
+        // flight at once, then expand it into the group's table.
         constexpr int span = 2 * KS - 1;
+        constexpr int PER = (C::RAW + 127) / 128;
+        float rv[PER];
+#pragma unroll
+        for (int m = 0; m < PER; ++m) {
+          const int idx = gtid + 128 * m;
+          rv[m] = (idx < C::RAW && rpb) ? to_f(rpb[(size_t)pr.h * C::RAW + idx]) * c : 0.f;
+        }
+#pragma unroll
+        for (int m = 0; m < PER; ++m)
+          if (gtid + 128 * m < C::RAW) raw[gtid + 128 * m] = rv[m];
+        named_barrier(1 + g, 128);  // raw is visible; the previous pair's table reads are done
         for (int idx = gtid; idx < C::TBL_ROWS * C::TBL_W; idx += 128) {
           const int row = idx / C::TBL_W, col = idx % C::TBL_W;
           const int blk = col / (KS + C::PAD), off = col % (KS + C::PAD);
           float v = -INFINITY;
-          if (row < span && blk < KS && off >= C::PAD) {
-            const int bc = blk + (off - C::PAD);
-            v = rpb ? to_f(rpb[((size_t)pr.h * span + row) * span + bc]) : 0.f;
-          }
+          if (row < span && blk < KS && off >= C::PAD) v = raw[row * span + blk + (off - C::PAD)];
           tbl[idx] = v;
         }
         named_barrier(1 + g, 128);
@@ -482,12 +567,12 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
       for (int cc = 0; cc < D; cc += 32) {
         uint32_t oa[32], ob[32];
-        tmem_ld32(sbuf + C::PO + cc, oa);
-        tmem_ld32(sbuf + C::PO + D + cc, ob);
+        tmem_ld32(obuf + cc, oa);
+        tmem_ld32(obuf + D + cc, ob);
         tmem_wait_ld();
         if (cc + 32 >= D) {
           tc_fence_before();
-          mbar_arrive(bar_o_empty(g));
+          mbar_arrive(bar_o_empty(C::SHARED_O ? 0 : g));
         }
         if (valid) {
 #pragma unroll
@@ -572,7 +657,14 @@ cudaError_t launch(const void* q, const void* k, const void* v, const void* rpb,
   {
     std::lock_guard<std::mutex> lk(mu);
     if (!attr_set[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+      // The run-time register split (setmaxnreg) must fit what the CTA is
+      // launched with, or its warpgroups would wait for registers forever.
+      cudaFuncAttributes fa;
+      cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+      if (e != cudaSuccess) return e;
+      if (C::NBUF == 2 && C::REGS_CTRL * 128 + C::REGS_SOFTMAX * 256 > fa.numRegs * C::THREADS)
+        return cudaErrorInvalidConfiguration;
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
       if (e != cudaSuccess) return e;
       attr_set[dev] = true;
     }
