@@ -58,7 +58,8 @@ struct Cfg {
   static constexpr int QBLK = 2 * TT * TT * ROWB;      // one K block of the query operand (128 rows)
   static constexpr int Q_BYTES = 2 * QBLK;
   static constexpr int KV_BYTES = HHP * HW * ROWB;
-  static constexpr int STAGE_BYTES = Q_BYTES + 2 * KV_BYTES;
+  static constexpr int QK_BYTES = Q_BYTES + KV_BYTES;  // one stage of the Q/K ring
+  static constexpr int STAGE_BYTES = QK_BYTES + KV_BYTES;  // plus one stage of the V ring
   // tensor memory: per buffer S (NS columns); P (16-bit) overlays its first
   // NS/2 columns; O (2d columns: tile A's d, then tile B's d) sits in the
   // dead part of S after P.
@@ -81,9 +82,19 @@ struct Cfg {
   static constexpr int TBL_W0 = KS * (KS + PAD) + PAD;
   static constexpr int TBL_W = TBL_W0 + ((8 - TBL_W0 % 32) + 32) % 32;  // = 8 mod 32: conflict-free rows
   static constexpr int TBL_ROWS = 2 * KS;
-  static constexpr int TBL_BYTES = TBL_ROWS * TBL_W * 4;
+  static constexpr int TBL_N = TBL_ROWS * TBL_W;
+  static_assert(TBL_W % 2 == 0, "table rows keep the parity of a column");
   static constexpr int RAW = (2 * KS - 1) * (2 * KS - 1);  // one head's bias table
   static constexpr int RAW_BYTES = round_up(RAW * 4, 16);
+  // With two copies of the table, the second shifted left by one entry,
+  // every lane reads its bias pairs with 8-byte loads from whichever copy
+  // makes them aligned.  The second copy is kept only where it costs no
+  // pipeline stage.
+  static constexpr int stages_with(int copies) {
+    return (kMaxSmem - (1024 + NBUF * (copies * TBL_N * 4 + RAW_BYTES) + 512)) / STAGE_BYTES;
+  }
+  static constexpr int TBL_COPIES = (stages_with(2) >= 3 || stages_with(2) == stages_with(1)) ? 2 : 1;
+  static constexpr int TBL_BYTES = TBL_COPIES * TBL_N * 4;
   static constexpr int FIXED = 1024 + NBUF * (TBL_BYTES + RAW_BYTES) + 512;  // + barriers, TMEM slot
   static constexpr int STAGES_FIT = (kMaxSmem - FIXED) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT >= 3 ? 3 : STAGES_FIT;
@@ -96,7 +107,8 @@ struct Cfg {
   // exactly the registers a 384-thread CTA is launched with (168 each).
   static constexpr int THREADS = 128 * (1 + NBUF);
   static constexpr int LAUNCH_REGS = 168;
-  static constexpr int REGS_CTRL = KS <= 5 ? 80 : 72, REGS_SOFTMAX = KS <= 5 ? 208 : 216;
+  static constexpr bool kWideCtrl = KS <= 5 || (D == 64 && KS > 9);
+  static constexpr int REGS_CTRL = kWideCtrl ? 80 : 72, REGS_SOFTMAX = kWideCtrl ? 208 : 216;
   static_assert(NBUF == 1 || REGS_CTRL * 128 + REGS_SOFTMAX * 256 <= LAUNCH_REGS * THREADS,
                 "the register split must fit the launch allocation");
   static constexpr uint32_t LAYOUT = ROWB == 64 ? kLayoutSW64 : kLayoutSW128;
@@ -234,11 +246,19 @@ template <> NA_DEVICE uint32_t exp2_pair<__nv_bfloat16>(float a0, float a1) {
   return ex2_bf16x2(pack2<__nv_bfloat16>(a0, a1));
 }
 template <> NA_DEVICE uint32_t exp2_pair<__half>(float a0, float a1) { return ex2_f16x2(pack2<__half>(a0, a1)); }
-template <typename T> NA_DEVICE float2 unpack2(uint32_t w);
-template <> NA_DEVICE float2 unpack2<__nv_bfloat16>(uint32_t w) {
-  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+// s0 += low half of w, s1 += high half, each taken exactly as a float (one
+// mixed-precision add per element, no unpacking).
+template <typename T> NA_DEVICE void acc_pair(float& s0, float& s1, uint32_t w);
+template <> NA_DEVICE void acc_pair<__nv_bfloat16>(float& s0, float& s1, uint32_t w) {
+  asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %2;\n add.rn.f32.bf16 %0, lo, %0;\n add.rn.f32.bf16 %1, hi, %1;\n}"
+      : "+f"(s0), "+f"(s1)
+      : "r"(w));
 }
-template <> NA_DEVICE float2 unpack2<__half>(uint32_t w) { return __half22float2(*reinterpret_cast<__half2*>(&w)); }
+template <> NA_DEVICE void acc_pair<__half>(float& s0, float& s1, uint32_t w) {
+  asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %2;\n add.rn.f32.f16 %0, lo, %0;\n add.rn.f32.f16 %1, hi, %1;\n}"
+      : "+f"(s0), "+f"(s1)
+      : "r"(w));
+}
 
 // Softmax of one warp's 32 queries (two 4x4 patches, one per tile) over the
 // union rows [u_r0, u_r1) and pieces [PB, PB+NU) of their windows, RB rows
@@ -251,8 +271,7 @@ template <> NA_DEVICE float2 unpack2<__half>(uint32_t w) { return __half22float2
 // sum of the rounded P.  Rows past u_r1 in the last batch repeat row u_r1-1:
 // they store the same values again and are left out of the sum.
 template <typename T, int KS, int D, int PB, int NU>
-NA_DEVICE float softmax_rows(uint32_t sbuf, const float* tbl, int u_r0, int u_r1, int wr0, int er, int colbase,
-                             float c) {
+NA_DEVICE float softmax_rows(uint32_t sbuf, const float* tl, int u_r0, int u_r1, int wr0, int er, float c) {
   using C = Cfg<KS, D>;
   constexpr int HW = C::HW, PW = HW / 2, NV = NU * 4, RB = 2;
   // start-column alignment of a piece window (row hr * HW + PB * 4) and of a P row (hr * PW)
@@ -271,13 +290,20 @@ NA_DEVICE float softmax_rows(uint32_t sbuf, const float* tbl, int u_r0, int u_r1
 #pragma unroll
     for (int j = 0; j < RB; ++j) {
       const int hr = min(r0 + j, last);
-      const float* tr =
-          tbl + ((unsigned)(hr - wr0) < (unsigned)KS ? hr + er : 2 * KS - 1) * C::TBL_W + colbase + PB * 4;
+      const float* tr = tl + ((unsigned)(hr - wr0) < (unsigned)KS ? hr + er : 2 * KS - 1) * C::TBL_W + PB * 4;
 #pragma unroll
       for (int e = 0; e < NV; e += 4) {
+        float2 b01, b23;
+        if constexpr (C::TBL_COPIES == 2) {
+          b01 = reinterpret_cast<const float2*>(tr)[e / 2];
+          b23 = reinterpret_cast<const float2*>(tr)[e / 2 + 1];
+        } else {
+          b01 = make_float2(tr[e], tr[e + 1]);
+          b23 = make_float2(tr[e + 2], tr[e + 3]);
+        }
         float y0, y1, y2, y3;
-        fma2(y0, y1, __uint_as_float(v[j][e]), __uint_as_float(v[j][e + 1]), c, c, tr[e], tr[e + 1]);
-        fma2(y2, y3, __uint_as_float(v[j][e + 2]), __uint_as_float(v[j][e + 3]), c, c, tr[e + 2], tr[e + 3]);
+        fma2(y0, y1, __uint_as_float(v[j][e]), __uint_as_float(v[j][e + 1]), c, c, b01.x, b01.y);
+        fma2(y2, y3, __uint_as_float(v[j][e + 2]), __uint_as_float(v[j][e + 3]), c, c, b23.x, b23.y);
         mx[j] = max3(mx[j], max3(y0, y1, y2), y3);
         v[j][e] = __float_as_uint(y0);
         v[j][e + 1] = __float_as_uint(y1);
@@ -315,9 +341,8 @@ NA_DEVICE float softmax_rows(uint32_t sbuf, const float* tbl, int u_r0, int u_r1
         add2(a0, a1, __uint_as_float(v[j][e]), __uint_as_float(v[j][e + 1]), -m, -m);
         add2(a2, a3, __uint_as_float(v[j][e + 2]), __uint_as_float(v[j][e + 3]), -m, -m);
         const uint32_t pa = exp2_pair<T>(a0, a1), pb = exp2_pair<T>(a2, a3);
-        const float2 fa = unpack2<T>(pa), fb = unpack2<T>(pb);
-        add2(s0, s1, s0, s1, fa.x, fa.y);
-        add2(s0, s1, s0, s1, fb.x, fb.y);
+        acc_pair<T>(s0, s1, pa);
+        acc_pair<T>(s0, s1, pb);
         pk[PB * 2 + e / 2] = pa;
         pk[PB * 2 + e / 2 + 1] = pb;
       }
@@ -333,15 +358,15 @@ NA_DEVICE float softmax_rows(uint32_t sbuf, const float* tbl, int u_r0, int u_r1
 // window union, fixed at compile time, or over whole rows when the union is
 // wider (patches at the map border).
 template <typename T, int KS, int D, int PB = 0>
-NA_DEVICE float softmax_dispatch(int pb, int pe, uint32_t sbuf, const float* tbl, int u_r0, int u_r1, int wr0,
-                                 int er, int colbase, float c) {
+NA_DEVICE float softmax_dispatch(int pb, int pe, uint32_t sbuf, const float* tl, int u_r0, int u_r1, int wr0,
+                                 int er, float c) {
   using C = Cfg<KS, D>;
   if constexpr (PB + C::NPU <= C::NPC) {
     if (pe - pb <= C::NPU && min(pb, C::NPC - C::NPU) == PB)
-      return softmax_rows<T, KS, D, PB, C::NPU>(sbuf, tbl, u_r0, u_r1, wr0, er, colbase, c);
-    return softmax_dispatch<T, KS, D, PB + 1>(pb, pe, sbuf, tbl, u_r0, u_r1, wr0, er, colbase, c);
+      return softmax_rows<T, KS, D, PB, C::NPU>(sbuf, tl, u_r0, u_r1, wr0, er, c);
+    return softmax_dispatch<T, KS, D, PB + 1>(pb, pe, sbuf, tl, u_r0, u_r1, wr0, er, c);
   } else {
-    return softmax_rows<T, KS, D, 0, C::NPC>(sbuf, tbl, u_r0, u_r1, wr0, er, colbase, c);
+    return softmax_rows<T, KS, D, 0, C::NPC>(sbuf, tl, u_r0, u_r1, wr0, er, c);
   }
 }
 
@@ -359,26 +384,33 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   float* raws = reinterpret_cast<float*>(smem + ST * C::STAGE_BYTES + NB * C::TBL_BYTES);
   uint64_t* bars =
       reinterpret_cast<uint64_t*>(smem + ST * C::STAGE_BYTES + NB * (C::TBL_BYTES + C::RAW_BYTES));
-  // barrier slots: full[ST][NB] empty[ST] s_full[NB] p_full[NB] o_full[NB] s_free[NB] o_empty[NO].
-  // A stage's "full" barrier is split by buffer: each is waited on by one
+  // Two shared-memory rings of ST stages: Q and K (released when S = Q K^T
+  // has read them) and V (released when P.V has read it), each fed by its
+  // own producer thread, so the next pairs' Q and K arrive while this
+  // pair's softmax runs.
+  // barrier slots: kfull[ST][NB] vfull[ST][NB] kempty[ST] vempty[ST]
+  //                s_full[NB] p_full[NB] o_full[NB] s_free[NB] o_empty[NO].
+  // A stage's "full" barriers are split by buffer: each is waited on by one
   // issuer only, one phase per use, so a parity wait can never see a phase
-  // of a pair that belongs to the other buffer.  Pair n uses full[n % ST][n % NB],
-  // for the (n / LCM)-th time.
+  // of a pair that belongs to the other buffer.  Pair n uses
+  // kfull[n % ST][n % NB] and vfull[n % ST][n % NB] for the (n / LCM)-th time.
   constexpr int LCM = (ST % NB == 0) ? ST : ST * NB;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + ST * NB + ST + 5 * NB);
+  constexpr int B0 = 2 * ST * NB + 2 * ST;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B0 + 5 * NB);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto bar = [&](int i) { return smem_addr(bars + i); };
-  auto bar_full = [&](int n) { return bar((n % ST) * NB + n % NB); };
-  auto bar_empty = [&](int s) { return bar(ST * NB + s); };
-  constexpr int B0 = ST * NB + ST;
+  auto bar_kfull = [&](int n) { return bar((n % ST) * NB + n % NB); };
+  auto bar_vfull = [&](int n) { return bar(ST * NB + (n % ST) * NB + n % NB); };
+  auto bar_kempty = [&](int s) { return bar(2 * ST * NB + s); };
+  auto bar_vempty = [&](int s) { return bar(2 * ST * NB + ST + s); };
   auto bar_s_full = [&](int b) { return bar(B0 + b); };
   auto bar_p_full = [&](int b) { return bar(B0 + NB + b); };
   auto bar_o_full = [&](int b) { return bar(B0 + 2 * NB + b); };
   auto bar_s_free = [&](int b) { return bar(B0 + 3 * NB + b); };
   auto bar_o_empty = [&](int o) { return bar(B0 + 4 * NB + o); };
-  auto q_smem = [&](int s) { return sbase + s * C::STAGE_BYTES; };
-  auto k_smem = [&](int s) { return sbase + s * C::STAGE_BYTES + C::Q_BYTES; };
-  auto v_smem = [&](int s) { return sbase + s * C::STAGE_BYTES + C::Q_BYTES + C::KV_BYTES; };
+  auto q_smem = [&](int s) { return sbase + s * C::QK_BYTES; };
+  auto k_smem = [&](int s) { return sbase + s * C::QK_BYTES + C::Q_BYTES; };
+  auto v_smem = [&](int s) { return sbase + ST * C::QK_BYTES + s * C::KV_BYTES; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // The query operand of S = Q K^T is block structured: K block 0 holds
@@ -386,11 +418,10 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   // (lanes 16-31); the other rows of each block stay zero.
   for (int s = 0; s < ST; ++s)
     for (int i = threadIdx.x; i < C::Q_BYTES / 16; i += blockDim.x)
-      reinterpret_cast<uint4*>(smem + s * C::STAGE_BYTES)[i] = make_uint4(0u, 0u, 0u, 0u);
+      reinterpret_cast<uint4*>(smem + s * C::QK_BYTES)[i] = make_uint4(0u, 0u, 0u, 0u);
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   if (threadIdx.x == 0) {
-    for (int i = 0; i < ST * NB; ++i) mbar_init(bar(i), 1);
-    for (int s = 0; s < ST; ++s) mbar_init(bar_empty(s), 1);
+    for (int i = 0; i < 2 * ST * NB + 2 * ST; ++i) mbar_init(bar(i), 1);
     for (int b = 0; b < NB; ++b) {
       mbar_init(bar_s_full(b), 1);
       mbar_init(bar_p_full(b), 128);
@@ -412,27 +443,33 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
   if (warp < 4) {
   if constexpr (NB == 2) regs_dec<C::REGS_CTRL>();
-  if (warp == 0) {
-    // ------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == 3) {
+    // ------------------------------------- TMA producers (Q/K ring; V ring)
+    const bool qk = warp == 0;
     if (lane == 0) {
       int n = 0;
       for (PairIter it(blockIdx.x, gridDim.x, p); it.valid(p); it.next(p), ++n) {
         const int s = n % ST;
-        if (!mbar_wait(bar_empty(s), ((n / ST) & 1) ^ 1, abort_flag, p.status)) break;
+        if (!mbar_wait(qk ? bar_kempty(s) : bar_vempty(s), ((n / ST) & 1) ^ 1, abort_flag, p.status)) break;
         const Pair pr = it.pair<KS>(p);
-        const uint32_t full = bar_full(n);
-        mbar_expect_tx(full, C::STAGE_BYTES - C::Q_BYTES / 2);
+        if (qk) {
+          const uint32_t full = bar_kfull(n);
+          mbar_expect_tx(full, C::Q_BYTES / 2 + C::KV_BYTES);
 #pragma unroll
-        for (int tile = 0; tile < 2; ++tile)
+          for (int tile = 0; tile < 2; ++tile)
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            tma_load_5d(q_smem(s) + tile * C::QBLK + (32 * q + 16 * tile) * C::ROWB, &tm_q, full, 0,
-                        pr.j0 + (q & 1) * PQ, pr.i0 + tile * TT + (q >> 1) * PQ, pr.h, pr.b);
-        tma_load_5d(k_smem(s), &tm_k, full, 0, pr.c0, pr.R0, pr.h, pr.b);
-        tma_load_5d(v_smem(s), &tm_v, full, 0, pr.c0, pr.R0, pr.h, pr.b);
+            for (int q = 0; q < 4; ++q)
+              tma_load_5d(q_smem(s) + tile * C::QBLK + (32 * q + 16 * tile) * C::ROWB, &tm_q, full, 0,
+                          pr.j0 + (q & 1) * PQ, pr.i0 + tile * TT + (q >> 1) * PQ, pr.h, pr.b);
+          tma_load_5d(k_smem(s), &tm_k, full, 0, pr.c0, pr.R0, pr.h, pr.b);
+        } else {
+          const uint32_t full = bar_vfull(n);
+          mbar_expect_tx(full, C::KV_BYTES);
+          tma_load_5d(v_smem(s), &tm_v, full, 0, pr.c0, pr.R0, pr.h, pr.b);
+        }
       }
       for (int e = 0; e < ST && !*abort_flag; ++e, ++n)
-        mbar_wait(bar_empty(n % ST), ((n / ST) & 1) ^ 1, abort_flag, p.status);
+        mbar_wait(qk ? bar_kempty(n % ST) : bar_vempty(n % ST), ((n / ST) & 1) ^ 1, abort_flag, p.status);
     }
     __syncwarp();
   } else if (warp <= NB) {
@@ -444,16 +481,16 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (lane == 0) {
       constexpr uint32_t idesc_pv = idesc_f16(kBF16, 128, 2 * D, true);
       // Stages are contiguous, so a stage's descriptor is the first one plus
-      // s * STAGE_BYTES / 16 in the start-address field.
+      // s * QK_BYTES / 16 in the start-address field.
       const uint64_t dq0 = smem_desc(q_smem(0), 16, 8 * C::ROWB, C::LAYOUT);
       const uint64_t dk0 = smem_desc(k_smem(0), 16, 8 * C::ROWB, C::LAYOUT);
-      constexpr uint64_t kStageDesc = C::STAGE_BYTES >> 4;
+      constexpr uint64_t kStageDesc = C::QK_BYTES >> 4;
       const uint32_t d = tmem + C::s_col(b), o = tmem + C::o_col(b);
       int n = b, use = 0;
       for (PairIter it(blockIdx.x + b * gridDim.x, NB * gridDim.x, p); it.valid(p); it.next(p), n += NB, ++use) {
         const Pair pr = it.pair<KS>(p);
         const int s = n % ST;
-        if (!mbar_wait(bar_full(n), (n / LCM) & 1, abort_flag, p.status)) break;
+        if (!mbar_wait(bar_kfull(n), (n / LCM) & 1, abort_flag, p.status)) break;
         // S of this buffer is free once the buffer's previous P.V has read P
         // and, when O overlays S, once that pair's epilogue has read O.
         if constexpr (C::SHARED_O) {
@@ -475,10 +512,12 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           for (int kk = 0; kk < D / 16; ++kk) mma_ss(d + n0, qB + kk * 2, kB + no + kk * 2, idesc, 1u);
         }
         mma_commit(bar_s_full(b));
+        mma_commit(bar_kempty(s));
 
         if (!mbar_wait(bar_p_full(b), use & 1, abort_flag, p.status)) break;
         // a shared O must have been read by the epilogue of the CTA's previous pair
         if (C::SHARED_O && !mbar_wait(bar_o_empty(0), (n & 1) ^ 1, abort_flag, p.status)) break;
+        if (!mbar_wait(bar_vfull(n), (n / LCM) & 1, abort_flag, p.status)) break;
         tc_fence_after();
         // B = [V_A | V_B]: two MN blocks of d columns, tile B's rows rB halo rows further on
         const uint64_t vd = smem_desc(v_smem(s), (uint32_t)(pr.rB * C::HW * C::ROWB), 8 * C::ROWB, C::LAYOUT);
@@ -487,7 +526,7 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
         for (int kk = 1; kk < C::NS / 16; ++kk) mma_ts(o, d + kk * 8, vd + kk * kstep, idesc_pv, 1u);
         mma_commit(bar_o_full(b));
-        mma_commit(bar_empty(s));
+        mma_commit(bar_vempty(s));
         if constexpr (C::SHARED_O) mma_commit(bar_s_free(b));
       }
     }
@@ -529,13 +568,20 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         for (int m = 0; m < PER; ++m)
           if (gtid + 128 * m < C::RAW) raw[gtid + 128 * m] = rv[m];
         named_barrier(1 + g, 128);  // raw is visible; the previous pair's table reads are done
-        for (int idx = gtid; idx < C::TBL_ROWS * C::TBL_W; idx += 128) {
-          const int row = idx / C::TBL_W, col = idx % C::TBL_W;
+        // one table column per thread; entry x of the second copy is entry x + 1 of the first
+        for (int col = gtid; col < C::TBL_W; col += 128) {
           const int blk = col / (KS + C::PAD), off = col % (KS + C::PAD);
-          float v = -INFINITY;
-          if (row < span && blk < KS && off >= C::PAD) v = raw[row * span + blk + (off - C::PAD)];
-          tbl[idx] = v;
+          const bool live = blk < KS && off >= C::PAD;
+          const int bc = blk + (off - C::PAD);
+#pragma unroll
+          for (int row = 0; row < C::TBL_ROWS; ++row) {
+            const float v = (live && row < span) ? raw[row * span + bc] : -INFINITY;
+            const int x = row * C::TBL_W + col;
+            tbl[x] = v;
+            if (C::TBL_COPIES == 2 && x > 0) tbl[C::TBL_N + x - 1] = v;
+          }
         }
+        if (C::TBL_COPIES == 2 && gtid == 0) tbl[2 * C::TBL_N - 1] = -INFINITY;
         named_barrier(1 + g, 128);
         cur_h = pr.h;
       }
@@ -554,7 +600,9 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
       if (!mbar_wait(bar_s_full(g), use & 1, abort_flag, p.status)) break;
       tc_fence_after();
-      const float l = softmax_dispatch<T, KS, D>(pb, pe, sbuf, tbl, u_r0, u_r1, wr0, er, colbase, c);
+      // this lane's table origin, in the copy where its pairs are 8-byte aligned
+      const float* tl = (C::TBL_COPIES == 2 && (colbase & 1)) ? tbl + C::TBL_N + colbase - 1 : tbl + colbase;
+      const float l = softmax_dispatch<T, KS, D>(pb, pe, sbuf, tl, u_r0, u_r1, wr0, er, c);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p_full(g));
