@@ -107,7 +107,7 @@ struct Cfg {
   // exactly the registers a 384-thread CTA is launched with (168 each).
   static constexpr int THREADS = 128 * (1 + NBUF);
   static constexpr int LAUNCH_REGS = 168;
-  static constexpr bool kWideCtrl = KS <= 5 || (D == 64 && KS > 9);
+  static constexpr bool kWideCtrl = D == 64 && KS > 9;
   static constexpr int REGS_CTRL = kWideCtrl ? 80 : 72, REGS_SOFTMAX = kWideCtrl ? 208 : 216;
   static_assert(NBUF == 1 || REGS_CTRL * 128 + REGS_SOFTMAX * 256 <= LAUNCH_REGS * THREADS,
                 "the register split must fit the launch allocation");
