@@ -159,8 +159,8 @@ class ClockSampler:
 
 def cpu_oracle_throughput(w, seconds, rows_per_call=None):
     """Times the fp64 oracle (all host threads) on a bounded sample of the
-    workload: whole (b, h) maps, repeated until `seconds` have passed or the
-    whole workload was done once if that takes longer."""
+    workload: passes over all (b, h) maps, or over as many as one pass of
+    about `seconds` allows, repeated until `seconds` have passed."""
     import oracle
     from vision_sliding_window_b200.inputs import workload_inputs
 
@@ -169,15 +169,20 @@ def cpu_oracle_throughput(w, seconds, rows_per_call=None):
     rpb = rpb.double().numpy()
     nthreads = oracle.max_threads()
     maps = w.B * w.heads
-    # calibrate on one map
+    # warm the thread pool on one map, then size the sample: whole passes over
+    # the workload (or over as many maps as fit), repeated until `seconds`
+    oracle.forward_rows(q, k, v, rpb, w.ks, 0, w.H, nthreads)
     t0 = time.perf_counter()
     oracle.forward_rows(q, k, v, rpb, w.ks, 0, w.H, nthreads)
     per_map = max(time.perf_counter() - t0, 1e-6)
     n_maps = max(1, min(maps, int(seconds / per_map)))
-    passes = max(1, int(seconds / (per_map * n_maps))) if n_maps == maps else 1
+    passes = 0
     t0 = time.perf_counter()
-    for _ in range(passes):
+    while True:
         oracle.forward_rows(q, k, v, rpb, w.ks, 0, n_maps * w.H, nthreads)
+        passes += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
     dt = time.perf_counter() - t0
     qn = passes * n_maps * w.H * w.W * w.ks * w.ks
     sample = (f"{passes} pass(es) over {n_maps} of {maps} (b, h) maps of {w.name} "
