@@ -59,7 +59,6 @@ struct Cfg {
   static constexpr int Q_BYTES = 2 * QBLK;
   static constexpr int KV_BYTES = HHP * HW * ROWB;
   static constexpr int QK_BYTES = Q_BYTES + KV_BYTES;  // one stage of the Q/K ring
-  static constexpr int STAGE_BYTES = QK_BYTES + KV_BYTES;  // plus one stage of the V ring
   // tensor memory: per buffer S (NS columns); P (16-bit) overlays its first
   // NS/2 columns; O (2d columns: tile A's d, then tile B's d) sits in the
   // dead part of S after P.
@@ -90,6 +89,12 @@ struct Cfg {
   // every lane reads its bias pairs with 8-byte loads from whichever copy
   // makes them aligned.  The second copy is kept only where it costs no
   // pipeline stage.
+  // A stage holds Q, K and V.  Where not even one such stage fits (large k
+  // with d = 64), V is loaded into the K slot once S = Q K^T has read K
+  // (KV_ALIAS): a stage is then Q and one K-or-V slot.
+  static constexpr int FULL_STAGE = QK_BYTES + KV_BYTES;
+  static constexpr bool KV_ALIAS = (kMaxSmem - (1024 + NBUF * (TBL_N * 4 + RAW_BYTES) + 512)) / FULL_STAGE < 1;
+  static constexpr int STAGE_BYTES = KV_ALIAS ? QK_BYTES : FULL_STAGE;
   static constexpr int stages_with(int copies) {
     return (kMaxSmem - (1024 + NBUF * (copies * TBL_N * 4 + RAW_BYTES) + 512)) / STAGE_BYTES;
   }
@@ -410,7 +415,7 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   auto bar_o_empty = [&](int o) { return bar(B0 + 4 * NB + o); };
   auto q_smem = [&](int s) { return sbase + s * C::QK_BYTES; };
   auto k_smem = [&](int s) { return sbase + s * C::QK_BYTES + C::Q_BYTES; };
-  auto v_smem = [&](int s) { return sbase + ST * C::QK_BYTES + s * C::KV_BYTES; };
+  auto v_smem = [&](int s) { return C::KV_ALIAS ? k_smem(s) : sbase + ST * C::QK_BYTES + s * C::KV_BYTES; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // The query operand of S = Q K^T is block structured: K block 0 holds
@@ -450,7 +455,13 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       int n = 0;
       for (PairIter it(blockIdx.x, gridDim.x, p); it.valid(p); it.next(p), ++n) {
         const int s = n % ST;
-        if (!mbar_wait(qk ? bar_kempty(s) : bar_vempty(s), ((n / ST) & 1) ^ 1, abort_flag, p.status)) break;
+        bool ok;
+        if constexpr (C::KV_ALIAS)  // Q/K: the slot's previous V is consumed; V: this pair's K is
+          ok = qk ? mbar_wait(bar_vempty(s), ((n / ST) & 1) ^ 1, abort_flag, p.status)
+                  : mbar_wait(bar_kempty(s), (n / ST) & 1, abort_flag, p.status);
+        else
+          ok = mbar_wait(qk ? bar_kempty(s) : bar_vempty(s), ((n / ST) & 1) ^ 1, abort_flag, p.status);
+        if (!ok) break;
         const Pair pr = it.pair<KS>(p);
         if (qk) {
           const uint32_t full = bar_kfull(n);
@@ -469,7 +480,8 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
       }
       for (int e = 0; e < ST && !*abort_flag; ++e, ++n)
-        mbar_wait(qk ? bar_kempty(n % ST) : bar_vempty(n % ST), ((n / ST) & 1) ^ 1, abort_flag, p.status);
+        mbar_wait((qk != C::KV_ALIAS) ? bar_kempty(n % ST) : bar_vempty(n % ST), ((n / ST) & 1) ^ 1, abort_flag,
+                  p.status);
     }
     __syncwarp();
   } else if (warp <= NB) {
@@ -747,9 +759,7 @@ cudaError_t launch_ks(const void* q, const void* k, const void* v, const void* r
     case 7: return launch<T, 7, D>(q, k, v, rpb, out, s, status, st);
     case 9: return launch<T, 9, D>(q, k, v, rpb, out, s, status, st);
     case 11: return launch<T, 11, D>(q, k, v, rpb, out, s, status, st);
-    case 13:
-      if constexpr (D == 32) return launch<T, 13, D>(q, k, v, rpb, out, s, status, st);
-      break;
+    case 13: return launch<T, 13, D>(q, k, v, rpb, out, s, status, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -760,7 +770,7 @@ bool forward_tc_supported(const Shape& s, na_dtype dt) {
   if (dt != NA_F16 && dt != NA_BF16) return false;
   if (s.d != 32 && s.d != 64) return false;
   if (s.ks < 3 || s.ks > 13 || (s.ks & 1) == 0) return false;
-  if (s.ks == 13 && s.d != 32) return false;  // S + O would exceed tensor memory
+
   return true;
 }
 
