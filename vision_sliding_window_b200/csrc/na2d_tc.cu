@@ -265,6 +265,22 @@ template <> NA_DEVICE void acc_pair<__half>(float& s0, float& s1, uint32_t w) {
       : "r"(w));
 }
 
+// A bounded meeting point of a fixed set of threads: an mbarrier that each
+// arrives on once per meeting, then waits for (with the kernel's time limit
+// and abort flag), so no thread can be left waiting by one that gave up.
+struct Meeting {
+  uint32_t bar;
+  uint32_t phase;
+  volatile int* abort_flag;
+  unsigned* status;
+  NA_DEVICE bool sync() {
+    mbar_arrive(bar);
+    const bool ok = mbar_wait(bar, phase, abort_flag, status);
+    phase ^= 1;
+    return ok;
+  }
+};
+
 // Softmax of one warp's 32 queries (two 4x4 patches, one per tile) over the
 // union rows [u_r0, u_r1) and pieces [PB, PB+NU) of their windows, RB rows
 // at a time: each batch's tensor-memory loads are issued together and the RB
@@ -401,7 +417,8 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   // kfull[n % ST][n % NB] and vfull[n % ST][n % NB] for the (n / LCM)-th time.
   constexpr int LCM = (ST % NB == 0) ? ST : ST * NB;
   constexpr int B0 = 2 * ST * NB + 2 * ST;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B0 + 5 * NB);
+  // then: the table meeting of each softmax group [NB]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B0 + 6 * NB);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto bar = [&](int i) { return smem_addr(bars + i); };
   auto bar_kfull = [&](int n) { return bar((n % ST) * NB + n % NB); };
@@ -413,6 +430,7 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   auto bar_o_full = [&](int b) { return bar(B0 + 2 * NB + b); };
   auto bar_s_free = [&](int b) { return bar(B0 + 3 * NB + b); };
   auto bar_o_empty = [&](int o) { return bar(B0 + 4 * NB + o); };
+  auto bar_tbl = [&](int g) { return bar(B0 + 5 * NB + g); };
   auto q_smem = [&](int s) { return sbase + s * C::QK_BYTES; };
   auto k_smem = [&](int s) { return sbase + s * C::QK_BYTES + C::Q_BYTES; };
   auto v_smem = [&](int s) { return C::KV_ALIAS ? k_smem(s) : sbase + ST * C::QK_BYTES + s * C::KV_BYTES; };
@@ -434,6 +452,7 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       mbar_init(bar_s_free(b), 1);
     }
     for (int o = 0; o < C::NO; ++o) mbar_init(bar_o_empty(o), 128);
+    for (int g = 0; g < NB; ++g) mbar_init(bar_tbl(g), 128);
     *abort_flag = 0;
     mbar_init_fence();
     tma_prefetch_desc(&tm_q);
@@ -561,6 +580,7 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const float c = p.scale_log2;
     const T* rpb = static_cast<const T*>(p.rpb);
     T* out = static_cast<T*>(p.out);
+    Meeting tmeet{bar_tbl(g), 0u, abort_flag, p.status};
     int cur_h = -1;
     int use = 0;
     for (PairIter it(blockIdx.x + g * gridDim.x, NB * gridDim.x, p); it.valid(p); it.next(p), ++use) {
@@ -579,7 +599,7 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
         for (int m = 0; m < PER; ++m)
           if (gtid + 128 * m < C::RAW) raw[gtid + 128 * m] = rv[m];
-        named_barrier(1 + g, 128);  // raw is visible; the previous pair's table reads are done
+        if (!tmeet.sync()) break;  // raw is visible; the previous pair's table reads are done
         // one table column per thread; entry x of the second copy is entry x + 1 of the first
         for (int col = gtid; col < C::TBL_W; col += 128) {
           const int blk = col / (KS + C::PAD), off = col % (KS + C::PAD);
@@ -594,7 +614,7 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           }
         }
         if (C::TBL_COPIES == 2 && gtid == 0) tbl[2 * C::TBL_N - 1] = -INFINITY;
-        named_barrier(1 + g, 128);
+        if (!tmeet.sync()) break;
         cur_h = pr.h;
       }
       const int i = pr.i0 + pr0, j = pr.j0 + pc0;
