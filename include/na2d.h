@@ -122,6 +122,33 @@ na_status na2d_forward_host(const void *q_host, const void *k_host, const void *
                             na_dtype dt, void *stream);
 
 /*
+ * na2d_forward_host without a workspace argument, for callers that cannot
+ * allocate device memory: for example a plugin whose host framework owns
+ * every device allocation, or a caller that must not enter the driver's
+ * allocator on its path.  The pages have no counterpart to this call; it is
+ * a convenience of this library.
+ *
+ * Instead of a caller's workspace it stages the inputs and the output in one
+ * fixed device array that the library reserves, NA2D_NOALLOC_SCRATCH_BYTES
+ * (64 MiB) on every device that loads the library, held until the process
+ * exits.  Shapes whose na2d_forward_host_workspace_bytes() exceeds that are
+ * rejected with NA_ERR_UNSUPPORTED; otherwise arguments, errors and results
+ * are those of na2d_forward_host.  The call allocates nothing.
+ *
+ * The first call on a device looks up the array's device address on that
+ * device (it must be the current device); make that first call before any
+ * stream capture.  All calls on a device share the one array: calls whose
+ * work overlaps on the GPU (different streams, or host threads) race and may
+ * return wrong results.  Each call writes everything it reads from the
+ * array, so the contents left by an earlier call do not matter.
+ */
+#define NA2D_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+na_status na2d_forward_host_noalloc(const void *q_host, const void *k_host, const void *v_host,
+                                    const void *rpb_host, void *out_host,
+                                    int B, int heads, int H, int W, int d, int ksize,
+                                    na_dtype dt, void *stream);
+
+/*
  * Which kernel na2d_forward launches for these arguments: 1 = tensor-core
  * (tcgen05/TMEM/TMA) kernel, 0 = SIMT kernel, negative = the arguments are
  * rejected (the negated na_status).  Host-only; enqueues nothing.

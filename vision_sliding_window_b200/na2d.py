@@ -23,7 +23,7 @@ _DT = {torch.float32: NA_F32, torch.float16: NA_F16, torch.bfloat16: NA_BF16}
 # Every exported symbol of include/na2d.h.
 EXPORTS = (
     "na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward",
-    "na2d_forward_host_workspace_bytes", "na2d_forward_host", "na2d_forward_kernel",
+    "na2d_forward_host_workspace_bytes", "na2d_forward_host", "na2d_forward_host_noalloc", "na2d_forward_kernel",
     "na2d_device_status", "na2d_debug_timeout_probe", "na_status_str",
 )
 
@@ -57,13 +57,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.na2d_forward_host_workspace_bytes.argtypes = [*shape, i]
         lib.na2d_forward_host_workspace_bytes.restype = sz
         lib.na2d_forward_host.argtypes = [vp, vp, vp, vp, vp, vp, sz, *shape, i, vp]
+        lib.na2d_forward_host_noalloc.argtypes = [vp, vp, vp, vp, vp, *shape, i, vp]
         lib.na2d_forward_kernel.argtypes = [*shape, i]
         lib.na2d_device_status.argtypes = [vp]
         lib.na2d_debug_timeout_probe.argtypes = [ctypes.c_uint, vp]
         lib.na_status_str.argtypes = [i]
         lib.na_status_str.restype = ctypes.c_char_p
         for name in ("na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward",
-                     "na2d_forward_host", "na2d_forward_kernel", "na2d_device_status",
+                     "na2d_forward_host", "na2d_forward_host_noalloc", "na2d_forward_kernel", "na2d_device_status",
                      "na2d_debug_timeout_probe"):
             getattr(lib, name).restype = i
         _lib = lib
@@ -173,6 +174,24 @@ def forward_host(q_host, k_host, v_host, rpb_host, out_host, ksize: int, workspa
         workspace.numel() * workspace.element_size(), B, heads, H, W, d, ksize, _DT[q_host.dtype], st),
         "na2d_forward_host")
     return out_host
+
+
+def forward_host_noalloc(q_host, k_host, v_host, rpb_host, out_host, ksize: int, stream=None):
+    """na2d_forward_host_noalloc: host tensors in and out, staged in the
+    library's own fixed device array, for callers that cannot allocate device
+    memory; shapes needing more than NOALLOC_SCRATCH_BYTES are rejected."""
+    B, heads, H, W, d = _dims(q_host)
+    for t in (q_host, k_host, v_host, out_host) + ((rpb_host,) if rpb_host is not None else ()):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("host buffers must be contiguous CPU tensors")
+    st = ctypes.c_void_p(stream.cuda_stream) if stream is not None else _stream()
+    _check(load_library().na2d_forward_host_noalloc(
+        _ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(rpb_host), _ptr(out_host), B, heads, H, W, d, ksize,
+        _DT[q_host.dtype], st), "na2d_forward_host_noalloc")
+    return out_host
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20  # NA2D_NOALLOC_SCRATCH_BYTES of include/na2d.h
 
 
 def forward_kernel(B, heads, H, W, d, ksize, dtype) -> int:
