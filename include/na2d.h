@@ -25,8 +25,9 @@
  * Ownership: the caller allocates and owns every buffer.  Device pointers
  * must point to device memory of the current CUDA device and be 16-byte
  * aligned.  The library allocates no memory in any call; it keeps only a
- * per-device status word (a static device variable) and encoded TMA
- * descriptors passed by value to its kernels.
+ * per-device status word (a static device variable), encoded TMA
+ * descriptors passed by value to its kernels, and the fixed staging array
+ * of na2d_forward_host_noalloc (a static device variable).
  *
  * Streams: every call that takes `stream` (a cudaStream_t passed as void*,
  * NULL meaning the legacy default stream) only enqueues work on it and
