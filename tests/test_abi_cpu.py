@@ -100,6 +100,19 @@ def test_forward_kernel_selection(lib):
         assert lib.na2d_forward_kernel(32, 2, 56, 56, 32, 7, dt) in (0, 1)
 
 
+def test_every_benchmarked_16_bit_workload_runs_on_the_tensor_core_kernel(lib):
+    from vision_sliding_window_b200.inputs import WORKLOADS
+
+    dts = {"f16": na2d.NA_F16, "bf16": na2d.NA_BF16}
+    for w in WORKLOADS.values():
+        if w.dtype in dts:
+            assert lib.na2d_forward_kernel(w.B, w.heads, w.H, w.W, w.d, w.ks, dts[w.dtype]) == 1, w.name
+    # every odd k from 3 to 13 at d = 32 and d = 64
+    for d in (32, 64):
+        for ks in range(3, 14, 2):
+            assert lib.na2d_forward_kernel(2, 2, 40, 40, d, ks, na2d.NA_BF16) == 1, (d, ks)
+
+
 def test_timeout_probe_rejects_bad_limits(lib):
     assert lib.na2d_debug_timeout_probe(0, None) == na2d.NA_ERR_INVALID_ARG
     assert lib.na2d_debug_timeout_probe(2_000_000, None) == na2d.NA_ERR_INVALID_ARG
