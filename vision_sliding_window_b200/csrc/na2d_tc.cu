@@ -50,6 +50,8 @@ template <int KS, int D>
 struct Cfg {
   static constexpr int HH = TT + KS - 1;               // halo rows of one tile
   static constexpr int HHP = 2 * TT + KS - 1;          // halo rows of the pair buffer
+  static constexpr int HS = TT + KS / 2;               // halo rows of a bottom single tile
+  static_assert(2 * HS == HHP, "two single-tile halos fill a pair buffer");
   static constexpr int HW = round_up(TT + KS - 1, 8);  // halo columns
   static constexpr int NS = HH * HW;                   // keys of one tile = S columns
   static constexpr int NPC = HW / 4;                   // 4-key pieces per halo row
@@ -126,67 +128,91 @@ struct Cfg {
   static_assert(SMEM_BYTES <= kMaxSmem, "shared memory");
 };
 
+// Division by a divisor fixed at launch: q = (umulhi(n, m) + n) >> s for
+// 0 <= n < 2^31, with s = ceil(log2 d) and m = ceil(2^(32+s) / d) - 2^32.
+struct FastDiv {
+  uint32_t d, m, s;
+  FastDiv() = default;
+  explicit FastDiv(uint32_t div) : d(div), m(0), s(0) {
+    while ((1ull << s) < div) ++s;
+    m = (uint32_t)((((1ull << (32 + s)) + div - 1) / div) - (1ull << 32));
+  }
+  NA_DEVICE int div(int n) const { return (int)((__umulhi((uint32_t)n, m) + (uint32_t)n) >> s); }
+};
+
+// Work units.  A map's rows are cut into pairs of 8x8 tiles stacked
+// vertically (16 rows).  Where the last tile row of a map is a single tile
+// (1 to 8 rows left over), that tile's clamped halo is only TT + KS/2 rows,
+// so two such single tiles -- of the same head, any maps and columns --
+// share one pair: each gets its own halo box, tile A's in buffer rows
+// [0, HS) and tile B's in [HHP - HS, HHP), which fill the pair's buffer
+// exactly.  Per head: the full pairs (column fastest, then pair row, then
+// batch), then the packed pairs of single tiles in (batch, column) order.
 struct Params {
   const void* rpb;  // [heads][2KS-1][2KS-1] or nullptr
   void* out;
   int B, heads, H, W;
-  int n_pr, n_pc, total;  // pair rows / columns per map, pairs in all
+  int n_pc, n_fpr;                   // tile columns; full pair rows per map
+  int full_per_head, singles_per_head, per_head, total;
+  FastDiv div_head, div_pc, div_fpr;
   float scale_log2;       // log2(e) / sqrt(d)
   unsigned* status;
 };
 
-// A pair of 8x8 tiles: rows [i0, i0+16), columns [j0, j0+8) of map (b, h).
-// Halo origin (R0, c0); tile B's windows start rB rows below R0.
+// One work unit: per tile t (0 = A, TMEM lanes 0-15 of each quarter; 1 = B,
+// lanes 16-31) the map b[t], first query row i0[t] and column j0[t], the
+// halo box origin (R0[t], c0[t]) and rt[t], the map row of the tile's
+// S-space row 0.  Tile B's S-space starts rB buffer rows into the halo.
 struct Pair {
-  int b, h, i0, j0, R0, c0, rB;
+  int h;
+  bool packed, has_b;
+  int b[2], i0[2], j0[2], c0[2], R0[2], rt[2];
+  int rB;
 };
 
-// Walks the pair indices t, t + stride, ... of one role.  Pair index order
-// is (head, batch, pair row, pair column), column fastest; the walk keeps
-// the four digits and adds the stride's digits with carries, so the loop
-// does no division.
-struct PairIter {
-  int t, pc, pr, b, h;            // current pair
-  int s0, s1, s2, s3, stride;     // the stride's digits
-  NA_DEVICE void digits(int x, const Params& p, int& d0, int& d1, int& d2, int& d3) {
-    d0 = x % p.n_pc;
-    x /= p.n_pc;
-    d1 = x % p.n_pr;
-    x /= p.n_pr;
-    d2 = x % p.B;
-    d3 = x / p.B;
+template <int KS>
+NA_DEVICE Pair decode_pair(int t, const Params& p) {
+  constexpr int HHP = 2 * TT + KS - 1, HS = TT + KS / 2;
+  Pair q;
+  q.h = p.div_head.div(t);
+  const int r = t - q.h * p.per_head;
+  if (r < p.full_per_head) {
+    const int rr = p.div_pc.div(r);
+    const int pc = r - rr * p.n_pc;
+    const int b = p.div_fpr.div(rr);
+    const int pr = rr - b * p.n_fpr;
+    q.packed = false;
+    q.has_b = true;
+    q.b[0] = q.b[1] = b;
+    q.i0[0] = pr * 2 * TT;
+    q.i0[1] = q.i0[0] + TT;
+    q.j0[0] = q.j0[1] = pc * TT;
+    q.R0[0] = q.R0[1] = window_start(q.i0[0], p.H, KS);
+    q.c0[0] = q.c0[1] = min(q.j0[0] - KS / 2, window_start(q.j0[0], p.W, KS));
+    q.rB = window_start(min(q.i0[1], p.H - 1), p.H, KS) - q.R0[0];  // 0 .. 8
+    q.rt[0] = q.R0[0];
+    q.rt[1] = q.R0[0] + q.rB;
+  } else {
+    const int u = r - p.full_per_head;
+    q.packed = true;
+    q.has_b = 2 * u + 1 < p.singles_per_head;
+#pragma unroll
+    for (int tl = 0; tl < 2; ++tl) {
+      const int sidx = q.has_b ? 2 * u + tl : 2 * u;  // a missing tile B repeats tile A
+      const int b = p.div_pc.div(sidx);
+      const int pc = sidx - b * p.n_pc;
+      q.b[tl] = b;
+      q.i0[tl] = p.n_fpr * 2 * TT;
+      q.j0[tl] = pc * TT;
+      q.R0[tl] = window_start(q.i0[tl], p.H, KS);
+      q.c0[tl] = min(q.j0[tl] - KS / 2, window_start(q.j0[tl], p.W, KS));
+    }
+    q.rB = TT;
+    q.rt[0] = q.R0[0];
+    q.rt[1] = q.R0[1] - (HHP - HS - TT);
   }
-  NA_DEVICE PairIter(int t0, int stride_, const Params& p) : t(t0), stride(stride_) {
-    digits(t0, p, pc, pr, b, h);
-    digits(stride_, p, s0, s1, s2, s3);
-  }
-  NA_DEVICE bool valid(const Params& p) const { return t < p.total; }
-  NA_DEVICE void next(const Params& p) {
-    t += stride;
-    pc += s0;
-    int c = pc >= p.n_pc;
-    pc -= c ? p.n_pc : 0;
-    pr += s1 + c;
-    c = pr >= p.n_pr;
-    pr -= c ? p.n_pr : 0;
-    b += s2 + c;
-    c = b >= p.B;
-    b -= c ? p.B : 0;
-    h += s3 + c;
-  }
-  template <int KS>
-  NA_DEVICE Pair pair(const Params& p) const {
-    Pair q;
-    q.b = b;
-    q.h = h;
-    q.i0 = pr * 2 * TT;
-    q.j0 = pc * TT;
-    q.R0 = window_start(q.i0, p.H, KS);
-    q.rB = window_start(min(q.i0 + TT, p.H - 1), p.H, KS) - q.R0;  // 0 .. 8
-    q.c0 = min(q.j0 - KS / 2, window_start(q.j0, p.W, KS));
-    return q;
-  }
-};
+  return q;
+}
 
 template <typename T> NA_DEVICE float to_f(T x);
 template <> NA_DEVICE float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -394,7 +420,8 @@ NA_DEVICE float softmax_dispatch(int pb, int pe, uint32_t sbuf, const float* tl,
 template <typename T, int KS, int D>
 __global__ void __launch_bounds__(Cfg<KS, D>::THREADS, 1)
 na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const Params p) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k1,
+                   const __grid_constant__ CUtensorMap tm_v1, const Params p) {
   using C = Cfg<KS, D>;
   constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr int NB = C::NBUF, ST = C::STAGES;
@@ -458,6 +485,8 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_k1);
+    tma_prefetch_desc(&tm_v1);
   }
   if (warp == 1) tmem_alloc(smem_addr(tmem_slot), kTmemCols);
   tc_fence_before();
@@ -472,7 +501,7 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const bool qk = warp == 0;
     if (lane == 0) {
       int n = 0;
-      for (PairIter it(blockIdx.x, gridDim.x, p); it.valid(p); it.next(p), ++n) {
+      for (int t = blockIdx.x; t < p.total; t += gridDim.x, ++n) {
         const int s = n % ST;
         bool ok;
         if constexpr (C::KV_ALIAS)  // Q/K: the slot's previous V is consumed; V: this pair's K is
@@ -481,7 +510,7 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         else
           ok = mbar_wait(qk ? bar_kempty(s) : bar_vempty(s), ((n / ST) & 1) ^ 1, abort_flag, p.status);
         if (!ok) break;
-        const Pair pr = it.pair<KS>(p);
+        const Pair pr = decode_pair<KS>(t, p);
         if (qk) {
           const uint32_t full = bar_kfull(n);
           mbar_expect_tx(full, C::Q_BYTES / 2 + C::KV_BYTES);
@@ -490,12 +519,24 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
             for (int q = 0; q < 4; ++q)
               tma_load_5d(q_smem(s) + tile * C::QBLK + (32 * q + 16 * tile) * C::ROWB, &tm_q, full, 0,
-                          pr.j0 + (q & 1) * PQ, pr.i0 + tile * TT + (q >> 1) * PQ, pr.h, pr.b);
-          tma_load_5d(k_smem(s), &tm_k, full, 0, pr.c0, pr.R0, pr.h, pr.b);
+                          pr.j0[tile] + (q & 1) * PQ, pr.i0[tile] + (q >> 1) * PQ, pr.h, pr.b[tile]);
+          if (pr.packed) {
+            tma_load_5d(k_smem(s), &tm_k1, full, 0, pr.c0[0], pr.R0[0], pr.h, pr.b[0]);
+            tma_load_5d(k_smem(s) + (C::HHP - C::HS) * C::HW * C::ROWB, &tm_k1, full, 0, pr.c0[1], pr.R0[1],
+                        pr.h, pr.b[1]);
+          } else {
+            tma_load_5d(k_smem(s), &tm_k, full, 0, pr.c0[0], pr.R0[0], pr.h, pr.b[0]);
+          }
         } else {
           const uint32_t full = bar_vfull(n);
           mbar_expect_tx(full, C::KV_BYTES);
-          tma_load_5d(v_smem(s), &tm_v, full, 0, pr.c0, pr.R0, pr.h, pr.b);
+          if (pr.packed) {
+            tma_load_5d(v_smem(s), &tm_v1, full, 0, pr.c0[0], pr.R0[0], pr.h, pr.b[0]);
+            tma_load_5d(v_smem(s) + (C::HHP - C::HS) * C::HW * C::ROWB, &tm_v1, full, 0, pr.c0[1], pr.R0[1],
+                        pr.h, pr.b[1]);
+          } else {
+            tma_load_5d(v_smem(s), &tm_v, full, 0, pr.c0[0], pr.R0[0], pr.h, pr.b[0]);
+          }
         }
       }
       for (int e = 0; e < ST && !*abort_flag; ++e, ++n)
@@ -518,8 +559,8 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       constexpr uint64_t kStageDesc = C::QK_BYTES >> 4;
       const uint32_t d = tmem + C::s_col(b), o = tmem + C::o_col(b);
       int n = b, use = 0;
-      for (PairIter it(blockIdx.x + b * gridDim.x, NB * gridDim.x, p); it.valid(p); it.next(p), n += NB, ++use) {
-        const Pair pr = it.pair<KS>(p);
+      for (int t = blockIdx.x + b * gridDim.x; t < p.total; t += NB * gridDim.x, n += NB, ++use) {
+        const Pair pr = decode_pair<KS>(t, p);
         const int s = n % ST;
         if (!mbar_wait(bar_kfull(n), (n / LCM) & 1, abort_flag, p.status)) break;
         // S of this buffer is free once the buffer's previous P.V has read P
@@ -570,8 +611,8 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int wq = warp & 3;        // lane quarter
     const int gtid = threadIdx.x - 128 - 128 * g;
     const int tile = lane >> 4, l16 = lane & 15;
-    const int pr0 = (wq >> 1) * PQ + tile * TT + (l16 >> 2);  // query row inside the pair
-    const int pc0 = (wq & 1) * PQ + (l16 & 3);                // query column inside the pair
+    const int pr0 = (wq >> 1) * PQ + (l16 >> 2);  // query row inside the tile
+    const int pc0 = (wq & 1) * PQ + (l16 & 3);    // query column inside the tile
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
     const uint32_t sbuf = tmem + lane_base + C::s_col(g);
     const uint32_t obuf = tmem + lane_base + C::o_col(g);
@@ -583,8 +624,8 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     Meeting tmeet{bar_tbl(g), 0u, abort_flag, p.status};
     int cur_h = -1;
     int use = 0;
-    for (PairIter it(blockIdx.x + g * gridDim.x, NB * gridDim.x, p); it.valid(p); it.next(p), ++use) {
-      const Pair pr = it.pair<KS>(p);
+    for (int t = blockIdx.x + g * gridDim.x; t < p.total; t += NB * gridDim.x, ++use) {
+      const Pair pr = decode_pair<KS>(t, p);
       if (pr.h != cur_h) {
         // New head: stage its bias (times log2e / sqrt(d)) with all loads in
         // flight at once, then expand it into the group's table.
@@ -617,12 +658,12 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         if (!tmeet.sync()) break;
         cur_h = pr.h;
       }
-      const int i = pr.i0 + pr0, j = pr.j0 + pc0;
-      const bool valid = i < p.H && j < p.W;
+      const int i = (tile ? pr.i0[1] : pr.i0[0]) + pr0, j = (tile ? pr.j0[1] : pr.j0[0]) + pc0;
+      const bool valid = i < p.H && j < p.W && (tile == 0 || pr.has_b);
       const int ic = min(i, p.H - 1), jc = min(j, p.W - 1);
       const int si = window_start(ic, p.H, KS), sj = window_start(jc, p.W, KS);
-      const int rt = pr.R0 + (tile ? pr.rB : 0);               // this tile's halo row origin
-      const int wr0 = si - rt, wc0 = sj - pr.c0;               // window origin in the tile halo
+      const int rt = tile ? pr.rt[1] : pr.rt[0];                // map row of this tile's S-space row 0
+      const int wr0 = si - rt, wc0 = sj - (tile ? pr.c0[1] : pr.c0[0]);  // window origin in S-space
       const int er = rt - ic + KS - 1;                         // bias row of halo row 0
       const int colbase = (sj - jc + KS - 1) * (KS + C::PAD) + C::PAD - wc0;
       const int u_r0 = __reduce_min_sync(0xffffffffu, wr0);
@@ -642,7 +683,7 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       // epilogue: O / l, rounded to T (tile A's columns, then tile B's)
       if (!mbar_wait(bar_o_full(g), use & 1, abort_flag, p.status)) break;
       tc_fence_after();
-      T* dst = out + ((((size_t)pr.b * p.heads + pr.h) * p.H + ic) * p.W + jc) * D;
+      T* dst = out + ((((size_t)(tile ? pr.b[1] : pr.b[0]) * p.heads + pr.h) * p.H + ic) * p.W + jc) * D;
       const float inv = 1.f / l;
 #pragma unroll
       for (int cc = 0; cc < D; cc += 32) {
@@ -725,9 +766,10 @@ cudaError_t launch(const void* q, const void* k, const void* v, const void* rpb,
                    unsigned* status, cudaStream_t st) {
   using C = Cfg<KS, D>;
   constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mk1, mv1;
   if (!make_map(&mq, q, s, bf16, PQ, PQ) || !make_map(&mk, k, s, bf16, C::HW, C::HHP) ||
-      !make_map(&mv, v, s, bf16, C::HW, C::HHP))
+      !make_map(&mv, v, s, bf16, C::HW, C::HHP) || !make_map(&mk1, k, s, bf16, C::HW, C::HS) ||
+      !make_map(&mv1, v, s, bf16, C::HW, C::HS))
     return cudaErrorInvalidValue;
   auto kern = na2d_fwd_tc_kernel<T, KS, D>;
   static std::mutex mu;
@@ -756,17 +798,30 @@ cudaError_t launch(const void* q, const void* k, const void* v, const void* rpb,
   p.heads = s.heads;
   p.H = s.H;
   p.W = s.W;
-  p.n_pr = (s.H + 2 * TT - 1) / (2 * TT);
+  // A last tile row of 1..8 rows is made of single tiles, packed two per
+  // pair; a last pair row of 9..15 rows stays a (ragged) pair.
   p.n_pc = (s.W + TT - 1) / TT;
-  const long long pairs = (long long)p.n_pr * p.n_pc * s.B * s.heads;
+  const int rem = s.H % (2 * TT);
+  const bool singles = rem > 0 && rem <= TT;
+  p.n_fpr = singles ? s.H / (2 * TT) : (s.H + 2 * TT - 1) / (2 * TT);
+  const long long full = (long long)s.B * p.n_fpr * p.n_pc;
+  const long long single = singles ? (long long)s.B * p.n_pc : 0;
+  const long long per_head = full + (single + 1) / 2;
+  const long long pairs = per_head * s.heads;
   if (pairs > 0x7fffffffLL) return cudaErrorInvalidValue;
+  p.full_per_head = (int)full;
+  p.singles_per_head = (int)single;
+  p.per_head = (int)per_head;
   p.total = (int)pairs;
+  p.div_head = FastDiv((uint32_t)per_head);
+  p.div_pc = FastDiv((uint32_t)p.n_pc);
+  p.div_fpr = FastDiv((uint32_t)(p.n_fpr > 0 ? p.n_fpr : 1));
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)s.d));
   p.status = status;
   const int sms = sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
   const int grid = p.total < sms ? p.total : sms;
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, p);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, mk1, mv1, p);
   return cudaGetLastError();
 }
 
