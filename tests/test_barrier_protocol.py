@@ -2,8 +2,9 @@
 random interleavings on the CPU.
 
 Each role of the kernel's CTA is a generator: the Q/K and V TMA producers,
-one MMA issuer per tensor-memory buffer, and one softmax warpgroup per
-buffer.  Every role waits and arrives exactly as the kernel does.  The
+one MMA issuer per tensor-memory buffer, one softmax warpgroup per buffer,
+and the epilogue warpgroup, which takes every pair in order and receives
+each pair's row sums through shared memory.  Every role waits and arrives exactly as the kernel does.  The
 asynchronous completions -- a TMA load landing, an MMA chain finishing --
 fire after random delays.  A barrier holds a completed-phase count, and a
 parity wait succeeds when the current phase's parity differs from the parity
@@ -13,13 +14,16 @@ waited for, as mbarrier.try_wait.parity does.  The model checks that:
     parity aliasing);
   * no shared-memory slot is overwritten while an MMA still reads it, and
     every MMA reads the pair it was meant for;
-  * no tensor-memory S, P or O buffer is reused while still in use;
+  * no tensor-memory S, P or O buffer is reused while still in use, and no
+    shared-memory row-sum slot is overwritten before the epilogue read it;
   * nothing deadlocks.
 
 This covers every combination the kernel builds: 1-3 stages, 1-2 buffers,
-O shared or overlaying S, and V sharing the K slot.  A last test plants the
-one protocol mistake met while building the kernel -- one "full" barrier per
-stage shared by both issuers -- and checks that the model catches it.
+O shared or overlaying S, and V sharing the K slot.  The last tests plant
+the two protocol mistakes met while building the kernel -- one "full"
+barrier per stage shared by both issuers, and one "O read" barrier for a
+shared O although the epilogue may lag a use behind -- and check that the
+model catches them.
 """
 import random
 
@@ -48,7 +52,7 @@ class ProtocolError(AssertionError):
     pass
 
 
-def simulate(stages, nbuf, shared_o, alias, npairs, seed, split_full=True):
+def simulate(stages, nbuf, shared_o, alias, npairs, seed, split_full=True, split_o_empty=True):
     rnd = random.Random(seed)
     lcm = stages if stages % nbuf == 0 else stages * nbuf
     # split_full: one Q/K and one V "full" barrier per (stage, buffer), as in the kernel
@@ -62,11 +66,18 @@ def simulate(stages, nbuf, shared_o, alias, npairs, seed, split_full=True):
     p_full = [Barrier(f"p_full{b}") for b in range(nbuf)]
     o_full = [Barrier(f"o_full{b}") for b in range(nbuf)]
     s_free = [Barrier(f"s_free{b}") for b in range(nbuf)]
-    o_empty = [Barrier(f"o_empty{o}") for o in range(1 if shared_o else nbuf)]
+    # O overlaying S: one o_empty per buffer.  A shared O: one per pair parity,
+    # since the epilogue may lag a buffer's softmax by a use
+    n_oe = (2 if split_o_empty else 1) if shared_o else nbuf
+    o_empty = [Barrier(f"o_empty{o}") for o in range(n_oe)]
+    o_empty_of = lambda n: o_empty[n % n_oe]                # o_empty pair n arrives on
+    o_slot = (lambda b: 0) if shared_o else (lambda b: b)
+    l_full = {(b, par): Barrier(f"l_full{b}{par}") for b in range(nbuf) for par in (0, 1)}
+    lsum = {}                                                # row sums in shared memory, per buffer and parity
 
     kslot, vslot = [None] * stages, [None] * stages          # pair held by each slot
     kreaders, vreaders = [set() for _ in range(stages)], [set() for _ in range(stages)]
-    S, O = [None] * nbuf, [None] * len(o_empty)              # pair held by each buffer
+    S, O = [None] * nbuf, [None] * (1 if shared_o else nbuf)  # pair held by each buffer
     events, clock, seq = [], [0], [0]
 
     def later(fn, delay=None):
@@ -136,7 +147,7 @@ def simulate(stages, nbuf, shared_o, alias, npairs, seed, split_full=True):
             while not p_full[b].try_wait(use):
                 yield
             if shared_o and n > 0:  # the previous pair's epilogue has read O
-                while not o_empty[0].try_wait(n - 1):
+                while not o_empty_of(n - 1).try_wait((n - 1) // n_oe):
                     yield
             while not vfull[fkey(n)].try_wait(fphase(n)):
                 yield
@@ -165,21 +176,34 @@ def simulate(stages, nbuf, shared_o, alias, npairs, seed, split_full=True):
             check(S[g] == n, f"softmax of pair {n} finds S of pair {S[g]}")
             for _ in range(rnd.randint(0, 15)):
                 yield
+            slot = (g, use & 1)
+            check(lsum.get(slot, "read") == "read", f"row sums of pair {n} overwrite unread ones")
+            lsum[slot] = n
+            l_full[slot].arrive()
             p_full[g].arrive()
-            while not o_full[g].try_wait(use):
+        yield "done"
+
+    def epilogue():
+        for n in range(npairs):
+            b, use = n % nbuf, n // nbuf
+            while not l_full[(b, use & 1)].try_wait(use >> 1):
                 yield
-            o = 0 if shared_o else g
+            check(lsum[(b, use & 1)] == n, f"epilogue of pair {n} reads the row sums of pair {lsum[(b, use & 1)]}")
+            lsum[(b, use & 1)] = "read"
+            while not o_full[b].try_wait(use):
+                yield
+            o = o_slot(b)
             check(O[o] == n, f"epilogue of pair {n} finds O of pair {O[o]}")
             O[o] = None
             if not shared_o:
-                S[g] = None
-            o_empty[o].arrive()
+                S[b] = None
+            o_empty_of(n).arrive()
             for _ in range(rnd.randint(0, 5)):
                 yield
         yield "done"
 
     roles = [qk_producer(), v_producer()] + [issuer(b) for b in range(nbuf)] + [softmax_group(g)
-                                                                                 for g in range(nbuf)]
+                                                                                 for g in range(nbuf)] + [epilogue()]
     done = [False] * len(roles)
     for _ in range(10 ** 6):
         if all(done):
@@ -211,3 +235,12 @@ def test_model_catches_a_full_barrier_shared_by_both_issuers():
     with pytest.raises(AssertionError):
         for seed in range(40):
             simulate(1, 2, True, False, 6, seed, split_full=False)
+
+
+def test_model_catches_a_single_o_empty_for_a_shared_o():
+    # one barrier for "the epilogue has read the shared O": the epilogue may lag
+    # the softmax of a buffer by a use, and the issuer's parity wait passes early
+    with pytest.raises(AssertionError):
+        for seed in range(200):
+            for npairs in (5, 8, 13):
+                simulate(3, 2, True, False, npairs, seed, split_o_empty=False)

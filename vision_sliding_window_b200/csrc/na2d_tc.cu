@@ -71,7 +71,9 @@ struct Cfg {
   // by the two buffers instead of overlaying S: S of a buffer's next pair
   // can then be computed as soon as P.V has consumed P, before the epilogue.
   static constexpr bool SHARED_O = NBUF == 2 && 2 * NS + 2 * D <= kTmemCols;
-  static constexpr int NO = SHARED_O ? 1 : NBUF;  // O buffers
+  // o_empty barriers: per buffer when O overlays S; for a shared O one per
+  // pair parity, since the epilogue may lag a buffer's next softmax
+  static constexpr int NO = SHARED_O ? 2 : NBUF;
   static constexpr int s_col(int b) { return SHARED_O ? b * NS : b * BUF_COLS; }
   static constexpr int o_col(int b) { return SHARED_O ? 2 * NS : b * BUF_COLS + PO; }
   // bias / mask table (one per softmax group): rows 0..2KS-2 hold bias rows,
@@ -87,6 +89,7 @@ struct Cfg {
   static_assert(TBL_W % 2 == 0, "table rows keep the parity of a column");
   static constexpr int RAW = (2 * KS - 1) * (2 * KS - 1);  // one head's bias table
   static constexpr int RAW_BYTES = round_up(RAW * 4, 16);
+  static constexpr int LSUM_BYTES = 2 * 128 * 4;  // row sums handed to the epilogue, per buffer and use parity
   // With two copies of the table, the second shifted left by one entry,
   // every lane reads its bias pairs with 8-byte loads from whichever copy
   // makes them aligned.  The second copy is kept only where it costs no
@@ -95,28 +98,30 @@ struct Cfg {
   // with d = 64), V is loaded into the K slot once S = Q K^T has read K
   // (KV_ALIAS): a stage is then Q and one K-or-V slot.
   static constexpr int FULL_STAGE = QK_BYTES + KV_BYTES;
-  static constexpr bool KV_ALIAS = (kMaxSmem - (1024 + NBUF * (TBL_N * 4 + RAW_BYTES) + 512)) / FULL_STAGE < 1;
+  static constexpr bool KV_ALIAS =
+      (kMaxSmem - (1024 + NBUF * (TBL_N * 4 + RAW_BYTES + LSUM_BYTES) + 512)) / FULL_STAGE < 1;
   static constexpr int STAGE_BYTES = KV_ALIAS ? QK_BYTES : FULL_STAGE;
   static constexpr int stages_with(int copies) {
-    return (kMaxSmem - (1024 + NBUF * (copies * TBL_N * 4 + RAW_BYTES) + 512)) / STAGE_BYTES;
+    return (kMaxSmem - (1024 + NBUF * (copies * TBL_N * 4 + RAW_BYTES + LSUM_BYTES) + 512)) / STAGE_BYTES;
   }
   static constexpr int TBL_COPIES = (stages_with(2) >= 3 || stages_with(2) == stages_with(1)) ? 2 : 1;
   static constexpr int TBL_BYTES = TBL_COPIES * TBL_N * 4;
-  static constexpr int FIXED = 1024 + NBUF * (TBL_BYTES + RAW_BYTES) + 512;  // + barriers, TMEM slot
+  static constexpr int FIXED = 1024 + NBUF * (TBL_BYTES + RAW_BYTES + LSUM_BYTES) + 512;  // + barriers, TMEM slot
   static constexpr int STAGES_FIT = (kMaxSmem - FIXED) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT >= 3 ? 3 : STAGES_FIT;
   static constexpr int SMEM_RAW = FIXED + STAGES * STAGE_BYTES;
   static constexpr int SMEM_BYTES = SMEM_RAW > kMinSmem ? SMEM_RAW : kMinSmem;
-  // warpgroup 0: TMA producer (warp 0), MMA issuer (warp 1), two idle warps;
-  // warpgroups 1..NBUF: softmax groups.  With two softmax groups the register
-  // file is re-split at run time: the control warpgroup keeps REGS_CTRL per
-  // thread, the softmax groups grow to REGS_SOFTMAX, which together use
-  // exactly the registers a 384-thread CTA is launched with (168 each).
-  static constexpr int THREADS = 128 * (1 + NBUF);
-  static constexpr int LAUNCH_REGS = 168;
+  // Warpgroup 0: TMA producers (warps 0 and 3) and MMA issuers (warps
+  // 1..NBUF); warpgroups 1..NBUF: softmax groups, one per buffer; the last
+  // warpgroup: the epilogue of every pair.  The register file is re-split at
+  // run time (setmaxnreg) within what the CTA is launched with.
+  static constexpr int THREADS = 128 * (2 + NBUF);
+  static constexpr int LAUNCH_REGS = NBUF == 2 ? 128 : 168;  // 65536 / THREADS in steps of 8
   static constexpr bool kWideCtrl = D == 64 && KS > 9;
-  static constexpr int REGS_CTRL = kWideCtrl ? 80 : 72, REGS_SOFTMAX = kWideCtrl ? 208 : 216;
-  static_assert(NBUF == 1 || REGS_CTRL * 128 + REGS_SOFTMAX * 256 <= LAUNCH_REGS * THREADS,
+  static constexpr int REGS_CTRL = NBUF == 2 ? 64 : (kWideCtrl ? 80 : 72);
+  static constexpr int REGS_EPI = NBUF == 2 ? 56 : 80;
+  static constexpr int REGS_SOFTMAX = NBUF == 2 ? 192 : 232;
+  static_assert(REGS_CTRL * 128 + REGS_EPI * 128 + REGS_SOFTMAX * 128 * NBUF <= LAUNCH_REGS * THREADS,
                 "the register split must fit the launch allocation");
   static constexpr uint32_t LAYOUT = ROWB == 64 ? kLayoutSW64 : kLayoutSW128;
   static_assert(NS <= BUF_COLS && PO + 2 * D <= BUF_COLS, "S, P and O of a buffer must fit in tensor memory");
@@ -430,8 +435,9 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const uint32_t sbase = smem_addr(smem);
   float* tables = reinterpret_cast<float*>(smem + ST * C::STAGE_BYTES);
   float* raws = reinterpret_cast<float*>(smem + ST * C::STAGE_BYTES + NB * C::TBL_BYTES);
+  float* lsums = reinterpret_cast<float*>(smem + ST * C::STAGE_BYTES + NB * (C::TBL_BYTES + C::RAW_BYTES));
   uint64_t* bars =
-      reinterpret_cast<uint64_t*>(smem + ST * C::STAGE_BYTES + NB * (C::TBL_BYTES + C::RAW_BYTES));
+      reinterpret_cast<uint64_t*>(smem + ST * C::STAGE_BYTES + NB * (C::TBL_BYTES + C::RAW_BYTES + C::LSUM_BYTES));
   // Two shared-memory rings of ST stages: Q and K (released when S = Q K^T
   // has read them) and V (released when P.V has read it), each fed by its
   // own producer thread, so the next pairs' Q and K arrive while this
@@ -445,7 +451,9 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   constexpr int LCM = (ST % NB == 0) ? ST : ST * NB;
   constexpr int B0 = 2 * ST * NB + 2 * ST;
   // then: the table meeting of each softmax group [NB]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B0 + 6 * NB);
+  // and l_full [NB][2]: row sums of a buffer's use posted for the epilogue,
+  // one barrier per use parity (a group may run one use ahead of the epilogue)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B0 + 8 * NB);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto bar = [&](int i) { return smem_addr(bars + i); };
   auto bar_kfull = [&](int n) { return bar((n % ST) * NB + n % NB); };
@@ -458,6 +466,7 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   auto bar_s_free = [&](int b) { return bar(B0 + 3 * NB + b); };
   auto bar_o_empty = [&](int o) { return bar(B0 + 4 * NB + o); };
   auto bar_tbl = [&](int g) { return bar(B0 + 5 * NB + g); };
+  auto bar_l_full = [&](int b, int par) { return bar(B0 + 6 * NB + 2 * b + par); };
   auto q_smem = [&](int s) { return sbase + s * C::QK_BYTES; };
   auto k_smem = [&](int s) { return sbase + s * C::QK_BYTES + C::Q_BYTES; };
   auto v_smem = [&](int s) { return C::KV_ALIAS ? k_smem(s) : sbase + ST * C::QK_BYTES + s * C::KV_BYTES; };
@@ -480,6 +489,7 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     for (int o = 0; o < C::NO; ++o) mbar_init(bar_o_empty(o), 128);
     for (int g = 0; g < NB; ++g) mbar_init(bar_tbl(g), 128);
+    for (int i = 0; i < 2 * NB; ++i) mbar_init(bar_l_full(i >> 1, i & 1), 128);
     *abort_flag = 0;
     mbar_init_fence();
     tma_prefetch_desc(&tm_q);
@@ -495,7 +505,7 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const uint32_t tmem = *tmem_slot;
 
   if (warp < 4) {
-  if constexpr (NB == 2) regs_dec<C::REGS_CTRL>();
+  regs_dec<C::REGS_CTRL>();
   if (warp == 0 || warp == 3) {
     // ------------------------------------- TMA producers (Q/K ring; V ring)
     const bool qk = warp == 0;
@@ -588,7 +598,8 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
         if (!mbar_wait(bar_p_full(b), use & 1, abort_flag, p.status)) break;
         // a shared O must have been read by the epilogue of the CTA's previous pair
-        if (C::SHARED_O && !mbar_wait(bar_o_empty(0), (n & 1) ^ 1, abort_flag, p.status)) break;
+        if (C::SHARED_O && n > 0 && !mbar_wait(bar_o_empty((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, p.status))
+          break;
         if (!mbar_wait(bar_vfull(n), (n / LCM) & 1, abort_flag, p.status)) break;
         tc_fence_after();
         // B = [V_A | V_B]: two MN blocks of d columns, tile B's rows rB halo rows further on
@@ -604,9 +615,9 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     __syncwarp();
   }
-  } else {
-    if constexpr (NB == 2) regs_inc<C::REGS_SOFTMAX>();
-    // ----------------------------------------- softmax groups + epilogue
+  } else if (warp < 4 + 4 * NB) {
+    regs_inc<C::REGS_SOFTMAX>();
+    // --------------------------------------------------------- softmax groups
     const int g = (warp - 4) >> 2;  // group = tensor-memory buffer
     const int wq = warp & 3;        // lane quarter
     const int gtid = threadIdx.x - 128 - 128 * g;
@@ -615,12 +626,10 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int pc0 = (wq & 1) * PQ + (l16 & 3);    // query column inside the tile
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
     const uint32_t sbuf = tmem + lane_base + C::s_col(g);
-    const uint32_t obuf = tmem + lane_base + C::o_col(g);
     float* tbl = tables + g * (C::TBL_BYTES / 4);
     float* raw = raws + g * (C::RAW_BYTES / 4);
     const float c = p.scale_log2;
     const T* rpb = static_cast<const T*>(p.rpb);
-    T* out = static_cast<T*>(p.out);
     Meeting tmeet{bar_tbl(g), 0u, abort_flag, p.status};
     int cur_h = -1;
     int use = 0;
@@ -659,7 +668,6 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         cur_h = pr.h;
       }
       const int i = (tile ? pr.i0[1] : pr.i0[0]) + pr0, j = (tile ? pr.j0[1] : pr.j0[0]) + pc0;
-      const bool valid = i < p.H && j < p.W && (tile == 0 || pr.has_b);
       const int ic = min(i, p.H - 1), jc = min(j, p.W - 1);
       const int si = window_start(ic, p.H, KS), sj = window_start(jc, p.W, KS);
       const int rt = tile ? pr.rt[1] : pr.rt[0];                // map row of this tile's S-space row 0
@@ -676,28 +684,51 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       // this lane's table origin, in the copy where its pairs are 8-byte aligned
       const float* tl = (C::TBL_COPIES == 2 && (colbase & 1)) ? tbl + C::TBL_N + colbase - 1 : tbl + colbase;
       const float l = softmax_dispatch<T, KS, D>(pb, pe, sbuf, tl, u_r0, u_r1, wr0, er, c);
+      // the row sum goes to the epilogue warpgroup through shared memory
+      lsums[(g * 2 + (use & 1)) * 128 + wq * 32 + lane] = l;
+      mbar_arrive(bar_l_full(g, use & 1));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p_full(g));
-
-      // epilogue: O / l, rounded to T (tile A's columns, then tile B's)
-      if (!mbar_wait(bar_o_full(g), use & 1, abort_flag, p.status)) break;
+    }
+  } else {
+    if constexpr (C::REGS_EPI < C::LAUNCH_REGS) regs_dec<C::REGS_EPI>();
+    // ------------------------------------------------------------ epilogue
+    // Every pair of the CTA in order: O / l, rounded to T, stored.  O holds
+    // tile A's d columns, then tile B's.
+    const int wq = warp & 3;
+    const int tile = lane >> 4, l16 = lane & 15;
+    const int pr0 = (wq >> 1) * PQ + (l16 >> 2);
+    const int pc0 = (wq & 1) * PQ + (l16 & 3);
+    const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+    T* out = static_cast<T*>(p.out);
+    int n = 0;
+    for (int t = blockIdx.x; t < p.total; t += gridDim.x, ++n) {
+      const int b = n % NB, use = n / NB;
+      const Pair pr = decode_pair<KS>(t, p);
+      const int i = (tile ? pr.i0[1] : pr.i0[0]) + pr0, j = (tile ? pr.j0[1] : pr.j0[0]) + pc0;
+      const bool valid = i < p.H && j < p.W && (tile == 0 || pr.has_b);
+      T* dst = out + ((((size_t)(tile ? pr.b[1] : pr.b[0]) * p.heads + pr.h) * p.H + min(i, p.H - 1)) * p.W +
+                      min(j, p.W - 1)) * D;
+      if (!mbar_wait(bar_l_full(b, use & 1), (use >> 1) & 1, abort_flag, p.status)) break;
+      const float inv = 1.f / lsums[(b * 2 + (use & 1)) * 128 + wq * 32 + lane];
+      if (!mbar_wait(bar_o_full(b), use & 1, abort_flag, p.status)) break;
       tc_fence_after();
-      T* dst = out + ((((size_t)(tile ? pr.b[1] : pr.b[0]) * p.heads + pr.h) * p.H + ic) * p.W + jc) * D;
-      const float inv = 1.f / l;
+      const uint32_t obuf = tmem + lane_base + C::o_col(b);
 #pragma unroll
-      for (int cc = 0; cc < D; cc += 32) {
-        uint32_t oa[32], ob[32];
-        tmem_ld32(obuf + cc, oa);
-        tmem_ld32(obuf + D + cc, ob);
-        tmem_wait_ld();
-        if (cc + 32 >= D) {
+      for (int cc = 0; cc < D; cc += 16) {
+        uint32_t oa[16], ob[16];
+        tmem_ld16(obuf + cc, oa);
+        tmem_ld16(obuf + D + cc, ob);
+        tmem_wait_ld_regs(oa);
+        tmem_wait_ld_regs(ob);
+        if (cc + 16 >= D) {
           tc_fence_before();
-          mbar_arrive(bar_o_empty(C::SHARED_O ? 0 : g));
+          mbar_arrive(bar_o_empty(C::SHARED_O ? (n & 1) : b));
         }
         if (valid) {
 #pragma unroll
-          for (int x = 0; x < 32; x += 8) {
+          for (int x = 0; x < 16; x += 8) {
             float f[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(tile ? ob[x + e] : oa[x + e]) * inv;
@@ -784,7 +815,7 @@ cudaError_t launch(const void* q, const void* k, const void* v, const void* rpb,
       cudaFuncAttributes fa;
       cudaError_t e = cudaFuncGetAttributes(&fa, kern);
       if (e != cudaSuccess) return e;
-      if (C::NBUF == 2 && C::REGS_CTRL * 128 + C::REGS_SOFTMAX * 256 > fa.numRegs * C::THREADS)
+      if (C::REGS_CTRL * 128 + C::REGS_EPI * 128 + C::REGS_SOFTMAX * 128 * C::NBUF > fa.numRegs * C::THREADS)
         return cudaErrorInvalidConfiguration;
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
       if (e != cudaSuccess) return e;
