@@ -87,15 +87,14 @@ NA_DEVICE void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::
 template <int N>
 NA_DEVICE void tmem_wait_ld_regs(uint32_t (&r)[N]) {
   static_assert(N % 4 == 0 && N <= 32, "register groups of 4");
-  if constexpr (N == 4) {
-    asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]));
-  } else {
 #pragma unroll
-    for (int q = 0; q < N; q += 8)
-      asm volatile("tcgen05.wait::ld.sync.aligned;"
-                   : "+r"(r[q]), "+r"(r[q + 1]), "+r"(r[q + 2]), "+r"(r[q + 3]), "+r"(r[q + 4]), "+r"(r[q + 5]),
-                     "+r"(r[q + 6]), "+r"(r[q + 7]));
-  }
+  for (int q = 0; q + 8 <= N; q += 8)
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[q]), "+r"(r[q + 1]), "+r"(r[q + 2]), "+r"(r[q + 3]), "+r"(r[q + 4]), "+r"(r[q + 5]),
+                   "+r"(r[q + 6]), "+r"(r[q + 7]));
+  if constexpr (N % 8 == 4)
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[N - 4]), "+r"(r[N - 3]), "+r"(r[N - 2]), "+r"(r[N - 1]));
 }
 NA_DEVICE void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
