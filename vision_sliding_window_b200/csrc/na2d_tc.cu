@@ -296,7 +296,15 @@ template <> NA_DEVICE void acc_pair<__half>(float& s0, float& s1, uint32_t w) {
       : "r"(w));
 }
 
-// A bounded meeting point of a fixed set of threads: an mbarrier that each
+// Arrives on `bar` once for the whole warp, after every lane's earlier
+// memory operations: the barrier counts warps, not threads, which keeps
+// shared-memory atomics off the hot path.
+NA_DEVICE void warp_arrive(uint32_t bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+// A bounded meeting point of a fixed set of warps: an mbarrier that each
 // arrives on once per meeting, then waits for (with the kernel's time limit
 // and abort flag), so no thread can be left waiting by one that gave up.
 struct Meeting {
@@ -305,7 +313,7 @@ struct Meeting {
   volatile int* abort_flag;
   unsigned* status;
   NA_DEVICE bool sync() {
-    mbar_arrive(bar);
+    warp_arrive(bar);
     const bool ok = mbar_wait(bar, phase, abort_flag, status);
     phase ^= 1;
     return ok;
@@ -333,6 +341,7 @@ NA_DEVICE float softmax_rows(uint32_t sbuf, const float* tl, int u_r0, int u_r1,
   float mx[RB];
 #pragma unroll
   for (int j = 0; j < RB; ++j) mx[j] = -INFINITY;
+#pragma unroll 1
   for (int r0 = u_r0; r0 < u_r1; r0 += RB) {
     uint32_t v[RB][NV];
 #pragma unroll
@@ -373,8 +382,10 @@ NA_DEVICE float softmax_rows(uint32_t sbuf, const float* tl, int u_r0, int u_r1,
   uint32_t z[PW];
 #pragma unroll
   for (int e = 0; e < PW; ++e) z[e] = 0u;
+#pragma unroll 1
   for (int hr = 0; hr < u_r0; ++hr) st_span<PW, AP>(sbuf + hr * PW, z);
   float l = 0.f;
+#pragma unroll 1
   for (int r0 = u_r0; r0 < u_r1; r0 += RB) {
     uint32_t v[RB][NV];
 #pragma unroll
@@ -402,6 +413,7 @@ NA_DEVICE float softmax_rows(uint32_t sbuf, const float* tl, int u_r0, int u_r1,
       if (r0 + j < u_r1) l += s0 + s1;
     }
   }
+#pragma unroll 1
   for (int hr = u_r1; hr < C::HH; ++hr) st_span<PW, AP>(sbuf + hr * PW, z);
   return l;
 }
@@ -483,13 +495,13 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     for (int i = 0; i < 2 * ST * NB + 2 * ST; ++i) mbar_init(bar(i), 1);
     for (int b = 0; b < NB; ++b) {
       mbar_init(bar_s_full(b), 1);
-      mbar_init(bar_p_full(b), 128);
+      mbar_init(bar_p_full(b), 4);  // barriers a warpgroup meets count its 4 warps
       mbar_init(bar_o_full(b), 1);
       mbar_init(bar_s_free(b), 1);
     }
-    for (int o = 0; o < C::NO; ++o) mbar_init(bar_o_empty(o), 128);
-    for (int g = 0; g < NB; ++g) mbar_init(bar_tbl(g), 128);
-    for (int i = 0; i < 2 * NB; ++i) mbar_init(bar_l_full(i >> 1, i & 1), 128);
+    for (int o = 0; o < C::NO; ++o) mbar_init(bar_o_empty(o), 4);
+    for (int g = 0; g < NB; ++g) mbar_init(bar_tbl(g), 4);
+    for (int i = 0; i < 2 * NB; ++i) mbar_init(bar_l_full(i >> 1, i & 1), 4);
     *abort_flag = 0;
     mbar_init_fence();
     tma_prefetch_desc(&tm_q);
@@ -686,10 +698,10 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const float l = softmax_dispatch<T, KS, D>(pb, pe, sbuf, tl, u_r0, u_r1, wr0, er, c);
       // the row sum goes to the epilogue warpgroup through shared memory
       lsums[(g * 2 + (use & 1)) * 128 + wq * 32 + lane] = l;
-      mbar_arrive(bar_l_full(g, use & 1));
+      warp_arrive(bar_l_full(g, use & 1));
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_p_full(g));
+      warp_arrive(bar_p_full(g));
     }
   } else {
     if constexpr (C::REGS_EPI < C::LAUNCH_REGS) regs_dec<C::REGS_EPI>();
@@ -724,7 +736,7 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tmem_wait_ld_regs(ob);
         if (cc + 16 >= D) {
           tc_fence_before();
-          mbar_arrive(bar_o_empty(C::SHARED_O ? (n & 1) : b));
+          warp_arrive(bar_o_empty(C::SHARED_O ? (n & 1) : b));
         }
         if (valid) {
 #pragma unroll
