@@ -153,6 +153,9 @@ struct FastDiv {
 // [0, HS) and tile B's in [HHP - HS, HHP), which fill the pair's buffer
 // exactly.  Per head: the full pairs (column fastest, then pair row, then
 // batch), then the packed pairs of single tiles in (batch, column) order.
+// Unit t is pair t / heads of head t % heads: with the head fastest, the
+// pairs a softmax group takes (2 x gridDim apart) keep one head, and its
+// bias table, whenever the head count divides 2 x gridDim.
 struct Params {
   const void* rpb;  // [heads][2KS-1][2KS-1] or nullptr
   void* out;
@@ -179,8 +182,8 @@ template <int KS>
 NA_DEVICE Pair decode_pair(int t, const Params& p) {
   constexpr int HHP = 2 * TT + KS - 1, HS = TT + KS / 2;
   Pair q;
-  q.h = p.div_head.div(t);
-  const int r = t - q.h * p.per_head;
+  const int r = p.div_head.div(t);  // the head varies fastest
+  q.h = t - r * p.heads;
   if (r < p.full_per_head) {
     const int rr = p.div_pc.div(r);
     const int pc = r - rr * p.n_pc;
@@ -856,7 +859,7 @@ cudaError_t launch(const void* q, const void* k, const void* v, const void* rpb,
   p.singles_per_head = (int)single;
   p.per_head = (int)per_head;
   p.total = (int)pairs;
-  p.div_head = FastDiv((uint32_t)per_head);
+  p.div_head = FastDiv((uint32_t)s.heads);
   p.div_pc = FastDiv((uint32_t)p.n_pc);
   p.div_fpr = FastDiv((uint32_t)(p.n_fpr > 0 ? p.n_fpr : 1));
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)s.d));
