@@ -4,7 +4,8 @@ random interleavings on the CPU.
 Each role of the kernel's CTA is a generator: the Q/K and V TMA producers,
 one MMA issuer per tensor-memory buffer, one softmax warpgroup per buffer,
 and the epilogue warpgroup, which takes every pair in order and receives
-each pair's row sums through shared memory.  Every role waits and arrives exactly as the kernel does.  The
+each pair's row sums through shared memory.  Every role waits and arrives
+exactly as the kernel does (a warpgroup's arrivals are one arrival here).  The
 asynchronous completions -- a TMA load landing, an MMA chain finishing --
 fire after random delays.  A barrier holds a completed-phase count, and a
 parity wait succeeds when the current phase's parity differs from the parity
@@ -19,11 +20,11 @@ waited for, as mbarrier.try_wait.parity does.  The model checks that:
   * nothing deadlocks.
 
 This covers every combination the kernel builds: 1-3 stages, 1-2 buffers,
-O shared or overlaying S, and V sharing the K slot.  The last tests plant
-the two protocol mistakes met while building the kernel -- one "full"
-barrier per stage shared by both issuers, and one "O read" barrier for a
-shared O although the epilogue may lag a use behind -- and check that the
-model catches them.
+and V sharing the K slot.  O overlays the dead part of its buffer's S.  The
+last tests plant two protocol mistakes -- one "full" barrier per stage
+shared by both issuers (met while building the kernel), and an epilogue that
+releases a buffer before reading its O -- and check that the model catches
+them.
 """
 import random
 
@@ -52,7 +53,7 @@ class ProtocolError(AssertionError):
     pass
 
 
-def simulate(stages, nbuf, shared_o, alias, npairs, seed, split_full=True, split_o_empty=True):
+def simulate(stages, nbuf, alias, npairs, seed, split_full=True, early_release=False):
     rnd = random.Random(seed)
     lcm = stages if stages % nbuf == 0 else stages * nbuf
     # split_full: one Q/K and one V "full" barrier per (stage, buffer), as in the kernel
@@ -65,19 +66,13 @@ def simulate(stages, nbuf, shared_o, alias, npairs, seed, split_full=True, split
     s_full = [Barrier(f"s_full{b}") for b in range(nbuf)]
     p_full = [Barrier(f"p_full{b}") for b in range(nbuf)]
     o_full = [Barrier(f"o_full{b}") for b in range(nbuf)]
-    s_free = [Barrier(f"s_free{b}") for b in range(nbuf)]
-    # O overlaying S: one o_empty per buffer.  A shared O: one per pair parity,
-    # since the epilogue may lag a buffer's softmax by a use
-    n_oe = (2 if split_o_empty else 1) if shared_o else nbuf
-    o_empty = [Barrier(f"o_empty{o}") for o in range(n_oe)]
-    o_empty_of = lambda n: o_empty[n % n_oe]                # o_empty pair n arrives on
-    o_slot = (lambda b: 0) if shared_o else (lambda b: b)
+    o_empty = [Barrier(f"o_empty{b}") for b in range(nbuf)]
     l_full = {(b, par): Barrier(f"l_full{b}{par}") for b in range(nbuf) for par in (0, 1)}
     lsum = {}                                                # row sums in shared memory, per buffer and parity
 
     kslot, vslot = [None] * stages, [None] * stages          # pair held by each slot
     kreaders, vreaders = [set() for _ in range(stages)], [set() for _ in range(stages)]
-    S, O = [None] * nbuf, [None] * (1 if shared_o else nbuf)  # pair held by each buffer
+    S, O = [None] * nbuf, [None] * nbuf                      # pair held by each buffer's S and O
     events, clock, seq = [], [0], [0]
 
     def later(fn, delay=None):
@@ -128,9 +123,8 @@ def simulate(stages, nbuf, shared_o, alias, npairs, seed, split_full=True, split
             while not kfull[fkey(n)].try_wait(fphase(n)):
                 yield
             check(kslot[s] == n, f"QK({n}) reads Q/K of pair {kslot[s]}")
-            if use > 0:  # S of this buffer is free
-                free = s_free[b] if shared_o else o_empty[b]
-                while not free.try_wait(use - 1):
+            if use > 0:  # the epilogue has read the buffer's O, which overlays S
+                while not o_empty[b].try_wait(use - 1):
                     yield
             check(S[b] is None, f"QK({n}) overwrites S of pair {S[b]}")
             kreaders[s].add(n)
@@ -138,6 +132,7 @@ def simulate(stages, nbuf, shared_o, alias, npairs, seed, split_full=True, split
 
             def qk_done(n=n, s=s, b=b):
                 check(kslot[s] == n, f"Q/K slot of pair {n} changed under QK")
+                check(O[b] is None, f"QK({n}) overwrites O of pair {O[b]} before the epilogue read it")
                 kreaders[s].discard(n)
                 S[b] = n
                 s_full[b].arrive()
@@ -146,26 +141,19 @@ def simulate(stages, nbuf, shared_o, alias, npairs, seed, split_full=True, split
 
             while not p_full[b].try_wait(use):
                 yield
-            if shared_o and n > 0:  # the previous pair's epilogue has read O
-                while not o_empty_of(n - 1).try_wait((n - 1) // n_oe):
-                    yield
             while not vfull[fkey(n)].try_wait(fphase(n)):
                 yield
             check(vslot[s] == n, f"PV({n}) reads V of pair {vslot[s]}")
-            o = 0 if shared_o else b
-            check(O[o] is None, f"PV({n}) overwrites O of pair {O[o]}")
+            check(S[b] == n, f"PV({n}) reads P of pair {S[b]}")
+            check(O[b] is None, f"PV({n}) overwrites O of pair {O[b]}")
             vreaders[s].add(n)
 
-            def pv_done(n=n, s=s, b=b, o=o):
+            def pv_done(n=n, s=s, b=b):
                 check(vslot[s] == n, f"V slot of pair {n} changed under PV")
                 vreaders[s].discard(n)
-                O[o] = n
-                if shared_o:
-                    S[b] = None
+                O[b] = n
                 o_full[b].arrive()
                 vempty[s].arrive()
-                if shared_o:
-                    s_free[b].arrive()
             later(pv_done, qk_time + rnd.randint(1, 10))
         yield "done"
 
@@ -192,12 +180,15 @@ def simulate(stages, nbuf, shared_o, alias, npairs, seed, split_full=True, split
             lsum[(b, use & 1)] = "read"
             while not o_full[b].try_wait(use):
                 yield
-            o = o_slot(b)
-            check(O[o] == n, f"epilogue of pair {n} finds O of pair {O[o]}")
-            O[o] = None
-            if not shared_o:
-                S[b] = None
-            o_empty_of(n).arrive()
+            if early_release:  # planted mistake: the buffer is released before O is read
+                o_empty[b].arrive()
+                for _ in range(rnd.randint(0, 20)):
+                    yield
+            check(O[b] == n, f"epilogue of pair {n} finds O of pair {O[b]}")
+            O[b] = None
+            S[b] = None
+            if not early_release:
+                o_empty[b].arrive()
             for _ in range(rnd.randint(0, 5)):
                 yield
         yield "done"
@@ -218,15 +209,14 @@ def simulate(stages, nbuf, shared_o, alias, npairs, seed, split_full=True, split
     raise ProtocolError("deadlock")
 
 
-COMBOS = [(st, nb, sh, al) for st in (1, 2, 3) for nb in (1, 2) for sh in ((False, True) if nb == 2 else (False,))
-          for al in (False, True)]
+COMBOS = [(st, nb, al) for st in (1, 2, 3) for nb in (1, 2) for al in (False, True)]
 
 
-@pytest.mark.parametrize("stages,nbuf,shared_o,alias", COMBOS)
-def test_protocol_under_random_interleavings(stages, nbuf, shared_o, alias):
-    for seed in range(40):
+@pytest.mark.parametrize("stages,nbuf,alias", COMBOS)
+def test_protocol_under_random_interleavings(stages, nbuf, alias):
+    for seed in range(60):
         for npairs in (1, 2, 3, 5, 8, 13):
-            simulate(stages, nbuf, shared_o, alias, npairs, seed * 100 + npairs)
+            simulate(stages, nbuf, alias, npairs, seed * 100 + npairs)
 
 
 def test_model_catches_a_full_barrier_shared_by_both_issuers():
@@ -234,13 +224,13 @@ def test_model_catches_a_full_barrier_shared_by_both_issuers():
     # second issuer's parity wait passes a phase early
     with pytest.raises(AssertionError):
         for seed in range(40):
-            simulate(1, 2, True, False, 6, seed, split_full=False)
+            simulate(1, 2, False, 6, seed, split_full=False)
 
 
-def test_model_catches_a_single_o_empty_for_a_shared_o():
-    # one barrier for "the epilogue has read the shared O": the epilogue may lag
-    # the softmax of a buffer by a use, and the issuer's parity wait passes early
+def test_model_catches_a_buffer_released_before_its_o_is_read():
+    # the epilogue arrives on o_empty before it has read O: the buffer's next
+    # S = Q K^T, which overwrites the columns O overlays, may then land first
     with pytest.raises(AssertionError):
         for seed in range(200):
-            for npairs in (5, 8, 13):
-                simulate(3, 2, True, False, npairs, seed, split_o_empty=False)
+            for npairs in (3, 5, 8):
+                simulate(2, 2, False, npairs, seed, early_release=True)

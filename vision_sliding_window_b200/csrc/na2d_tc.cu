@@ -67,15 +67,8 @@ struct Cfg {
   static constexpr int NBUF = NS <= kTmemCols / 2 ? 2 : 1;
   static constexpr int BUF_COLS = kTmemCols / NBUF;
   static constexpr int PO = round_up(NS / 2, 32);
-  // When two S buffers and one O (2d columns) fit side by side, O is shared
-  // by the two buffers instead of overlaying S: S of a buffer's next pair
-  // can then be computed as soon as P.V has consumed P, before the epilogue.
-  static constexpr bool SHARED_O = NBUF == 2 && 2 * NS + 2 * D <= kTmemCols;
-  // o_empty barriers: per buffer when O overlays S; for a shared O one per
-  // pair parity, since the epilogue may lag a buffer's next softmax
-  static constexpr int NO = SHARED_O ? 2 : NBUF;
-  static constexpr int s_col(int b) { return SHARED_O ? b * NS : b * BUF_COLS; }
-  static constexpr int o_col(int b) { return SHARED_O ? 2 * NS : b * BUF_COLS + PO; }
+  static constexpr int s_col(int b) { return b * BUF_COLS; }
+  static constexpr int o_col(int b) { return b * BUF_COLS + PO; }
   // bias / mask table (one per softmax group): rows 0..2KS-2 hold bias rows,
   // row 2KS-1 is all -inf.  A row is KS blocks of stride KS+PAD; block dc
   // holds the bias row's columns dc..dc+KS-1 after PAD entries of -inf, and
@@ -125,7 +118,6 @@ struct Cfg {
                 "the register split must fit the launch allocation");
   static constexpr uint32_t LAYOUT = ROWB == 64 ? kLayoutSW64 : kLayoutSW128;
   static_assert(NS <= BUF_COLS && PO + 2 * D <= BUF_COLS, "S, P and O of a buffer must fit in tensor memory");
-  static_assert(!SHARED_O || NS % 32 == 0, "buffers start on 32-column boundaries");
   static_assert(STAGES >= 1, "a pipeline stage must fit in shared memory");
   static_assert(NS % 16 == 0, "halo keys must be a multiple of the MMA K step");
   static_assert(QBLK % 1024 == 0 && KV_BYTES % 1024 == 0 && (TT * HW * ROWB) % 1024 == 0,
@@ -458,7 +450,7 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   // own producer thread, so the next pairs' Q and K arrive while this
   // pair's softmax runs.
   // barrier slots: kfull[ST][NB] vfull[ST][NB] kempty[ST] vempty[ST]
-  //                s_full[NB] p_full[NB] o_full[NB] s_free[NB] o_empty[NO].
+  //                s_full[NB] p_full[NB] o_full[NB] o_empty[NB].
   // A stage's "full" barriers are split by buffer: each is waited on by one
   // issuer only, one phase per use, so a parity wait can never see a phase
   // of a pair that belongs to the other buffer.  Pair n uses
@@ -468,7 +460,7 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   // then: the table meeting of each softmax group [NB]
   // and l_full [NB][2]: row sums of a buffer's use posted for the epilogue,
   // one barrier per use parity (a group may run one use ahead of the epilogue)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B0 + 8 * NB);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B0 + 7 * NB);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto bar = [&](int i) { return smem_addr(bars + i); };
   auto bar_kfull = [&](int n) { return bar((n % ST) * NB + n % NB); };
@@ -478,10 +470,9 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   auto bar_s_full = [&](int b) { return bar(B0 + b); };
   auto bar_p_full = [&](int b) { return bar(B0 + NB + b); };
   auto bar_o_full = [&](int b) { return bar(B0 + 2 * NB + b); };
-  auto bar_s_free = [&](int b) { return bar(B0 + 3 * NB + b); };
-  auto bar_o_empty = [&](int o) { return bar(B0 + 4 * NB + o); };
-  auto bar_tbl = [&](int g) { return bar(B0 + 5 * NB + g); };
-  auto bar_l_full = [&](int b, int par) { return bar(B0 + 6 * NB + 2 * b + par); };
+  auto bar_o_empty = [&](int b) { return bar(B0 + 3 * NB + b); };
+  auto bar_tbl = [&](int g) { return bar(B0 + 4 * NB + g); };
+  auto bar_l_full = [&](int b, int par) { return bar(B0 + 5 * NB + 2 * b + par); };
   auto q_smem = [&](int s) { return sbase + s * C::QK_BYTES; };
   auto k_smem = [&](int s) { return sbase + s * C::QK_BYTES + C::Q_BYTES; };
   auto v_smem = [&](int s) { return C::KV_ALIAS ? k_smem(s) : sbase + ST * C::QK_BYTES + s * C::KV_BYTES; };
@@ -500,9 +491,8 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       mbar_init(bar_s_full(b), 1);
       mbar_init(bar_p_full(b), 4);  // barriers a warpgroup meets count its 4 warps
       mbar_init(bar_o_full(b), 1);
-      mbar_init(bar_s_free(b), 1);
+      mbar_init(bar_o_empty(b), 4);
     }
-    for (int o = 0; o < C::NO; ++o) mbar_init(bar_o_empty(o), 4);
     for (int g = 0; g < NB; ++g) mbar_init(bar_tbl(g), 4);
     for (int i = 0; i < 2 * NB; ++i) mbar_init(bar_l_full(i >> 1, i & 1), 4);
     *abort_flag = 0;
@@ -588,13 +578,9 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const Pair pr = decode_pair<KS>(t, p);
         const int s = n % ST;
         if (!mbar_wait(bar_kfull(n), (n / LCM) & 1, abort_flag, p.status)) break;
-        // S of this buffer is free once the buffer's previous P.V has read P
-        // and, when O overlays S, once that pair's epilogue has read O.
-        if constexpr (C::SHARED_O) {
-          if (!mbar_wait(bar_s_free(b), (use & 1) ^ 1, abort_flag, p.status)) break;
-        } else {
-          if (!mbar_wait(bar_o_empty(b), (use & 1) ^ 1, abort_flag, p.status)) break;
-        }
+        // S of this buffer is free once the epilogue has read the buffer's
+        // previous O, which overlays the dead part of S (after P.V read P).
+        if (!mbar_wait(bar_o_empty(b), (use & 1) ^ 1, abort_flag, p.status)) break;
         tc_fence_after();
         const uint64_t qA = dq0 + s * kStageDesc, qB = qA + (C::QBLK >> 4);
         const uint64_t kA = dk0 + s * kStageDesc, kB = kA + (uint64_t)(pr.rB * C::HW * C::ROWB >> 4);
@@ -612,9 +598,6 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         mma_commit(bar_kempty(s));
 
         if (!mbar_wait(bar_p_full(b), use & 1, abort_flag, p.status)) break;
-        // a shared O must have been read by the epilogue of the CTA's previous pair
-        if (C::SHARED_O && n > 0 && !mbar_wait(bar_o_empty((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, p.status))
-          break;
         if (!mbar_wait(bar_vfull(n), (n / LCM) & 1, abort_flag, p.status)) break;
         tc_fence_after();
         // B = [V_A | V_B]: two MN blocks of d columns, tile B's rows rB halo rows further on
@@ -625,7 +608,6 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         for (int kk = 1; kk < C::NS / 16; ++kk) mma_ts(o, d + kk * 8, vd + kk * kstep, idesc_pv, 1u);
         mma_commit(bar_o_full(b));
         mma_commit(bar_vempty(s));
-        if constexpr (C::SHARED_O) mma_commit(bar_s_free(b));
       }
     }
     __syncwarp();
@@ -739,7 +721,7 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tmem_wait_ld_regs(ob);
         if (cc + 16 >= D) {
           tc_fence_before();
-          warp_arrive(bar_o_empty(C::SHARED_O ? (n & 1) : b));
+          warp_arrive(bar_o_empty(b));
         }
         if (valid) {
 #pragma unroll
