@@ -69,36 +69,43 @@ struct Cfg {
   static constexpr int PO = round_up(NS / 2, 32);
   static constexpr int s_col(int b) { return b * BUF_COLS; }
   static constexpr int o_col(int b) { return b * BUF_COLS + PO; }
-  // bias / mask table (one per softmax group): rows 0..2KS-2 hold bias rows,
-  // row 2KS-1 is all -inf.  A row is KS blocks of stride KS+PAD; block dc
-  // holds the bias row's columns dc..dc+KS-1 after PAD entries of -inf, and
-  // its tail is the next block's -inf head.  PAD covers a whole halo row
-  // around any window.
+  // bias / mask table (one per softmax group), 16-bit entries of the input
+  // type, exactly the bias values given: rows 0..2KS-2 hold bias rows, row
+  // 2KS-1 is all -inf.  A row is KS blocks of stride KS+PAD; block dc holds
+  // the bias row's columns dc..dc+KS-1 after PAD entries of -inf, and its
+  // tail is the next block's -inf head.  PAD covers a whole halo row around
+  // any window.
   static constexpr int PAD = HW - KS;
   static constexpr int TBL_W0 = KS * (KS + PAD) + PAD;
-  static constexpr int TBL_W = TBL_W0 + ((8 - TBL_W0 % 32) + 32) % 32;  // = 8 mod 32: conflict-free rows
+  static constexpr int TBL_W = TBL_W0 + ((4 - TBL_W0 % 64) + 64) % 64;  // = 4 mod 64 entries
   static constexpr int TBL_ROWS = 2 * KS;
-  static constexpr int TBL_N = TBL_ROWS * TBL_W;
-  static_assert(TBL_W % 2 == 0, "table rows keep the parity of a column");
+  static constexpr int TBL_N = TBL_ROWS * TBL_W;  // entries of one copy
+  static_assert(TBL_W % 4 == 0 && TBL_N % 4 == 0, "table rows keep a column's offset mod 4");
+  // Copies of the table, copy q shifted left by q entries: every lane reads
+  // its entries 4 at a time with 8-byte loads (2 at a time with 4-byte loads
+  // when only two copies are kept) from the copy that makes them aligned.
+  // Copy q starts tbl_off(q) entries past a 64-entry boundary: offsets that
+  // spread the 16 lanes of a tile over distinct banks for the softmax's
+  // lane-to-query layout.  Four copies are kept where they cost no stage.
+  static constexpr int TBL_CS = round_up(TBL_N, 64);
+  static constexpr int tbl_off(int q) { return q == 0 ? 0 : q == 1 ? 16 : KS % 4 == 1 ? 16 * q : 16 * q + 4; }
+  static constexpr int tbl_base(int q) { return q * TBL_CS + tbl_off(q); }
+  static constexpr int tbl_bytes(int copies) { return round_up((tbl_base(copies - 1) + TBL_N) * 2, 16); }
   static constexpr int RAW = (2 * KS - 1) * (2 * KS - 1);  // one head's bias table
-  static constexpr int RAW_BYTES = round_up(RAW * 4, 16);
+  static constexpr int RAW_BYTES = round_up(RAW * 2, 16);
   static constexpr int LSUM_BYTES = 2 * 128 * 4;  // row sums handed to the epilogue, per buffer and use parity
-  // With two copies of the table, the second shifted left by one entry,
-  // every lane reads its bias pairs with 8-byte loads from whichever copy
-  // makes them aligned.  The second copy is kept only where it costs no
-  // pipeline stage.
   // A stage holds Q, K and V.  Where not even one such stage fits (large k
   // with d = 64), V is loaded into the K slot once S = Q K^T has read K
   // (KV_ALIAS): a stage is then Q and one K-or-V slot.
   static constexpr int FULL_STAGE = QK_BYTES + KV_BYTES;
   static constexpr bool KV_ALIAS =
-      (kMaxSmem - (1024 + NBUF * (TBL_N * 4 + RAW_BYTES + LSUM_BYTES) + 512)) / FULL_STAGE < 1;
+      (kMaxSmem - (1024 + NBUF * (tbl_bytes(2) + RAW_BYTES + LSUM_BYTES) + 512)) / FULL_STAGE < 1;
   static constexpr int STAGE_BYTES = KV_ALIAS ? QK_BYTES : FULL_STAGE;
   static constexpr int stages_with(int copies) {
-    return (kMaxSmem - (1024 + NBUF * (copies * TBL_N * 4 + RAW_BYTES + LSUM_BYTES) + 512)) / STAGE_BYTES;
+    return (kMaxSmem - (1024 + NBUF * (tbl_bytes(copies) + RAW_BYTES + LSUM_BYTES) + 512)) / STAGE_BYTES;
   }
-  static constexpr int TBL_COPIES = (stages_with(2) >= 3 || stages_with(2) == stages_with(1)) ? 2 : 1;
-  static constexpr int TBL_BYTES = TBL_COPIES * TBL_N * 4;
+  static constexpr int TBL_COPIES = (stages_with(4) >= 3 || stages_with(4) == stages_with(2)) ? 4 : 2;
+  static constexpr int TBL_BYTES = tbl_bytes(TBL_COPIES);
   static constexpr int FIXED = 1024 + NBUF * (TBL_BYTES + RAW_BYTES + LSUM_BYTES) + 512;  // + barriers, TMEM slot
   static constexpr int STAGES_FIT = (kMaxSmem - FIXED) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT >= 3 ? 3 : STAGES_FIT;
@@ -214,10 +221,6 @@ NA_DEVICE Pair decode_pair(int t, const Params& p) {
   return q;
 }
 
-template <typename T> NA_DEVICE float to_f(T x);
-template <> NA_DEVICE float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
-template <> NA_DEVICE float to_f(__half x) { return __half2float(x); }
-
 template <typename T> NA_DEVICE uint32_t pack2(float lo, float hi);
 template <> NA_DEVICE uint32_t pack2<__nv_bfloat16>(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -291,6 +294,25 @@ template <> NA_DEVICE void acc_pair<__half>(float& s0, float& s1, uint32_t w) {
       : "r"(w));
 }
 
+// d0 = s0 + low half of w, d1 = s1 + high half, each half taken exactly as
+// a float (mixed-precision adds, no unpacking).
+template <typename T> NA_DEVICE void add_pair(float& d0, float& d1, float s0, float s1, uint32_t w);
+template <> NA_DEVICE void add_pair<__nv_bfloat16>(float& d0, float& d1, float s0, float s1, uint32_t w) {
+  asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %2;\n add.rn.f32.bf16 %0, lo, %3;\n add.rn.f32.bf16 %1, hi, %4;\n}"
+      : "=f"(d0), "=f"(d1)
+      : "r"(w), "f"(s0), "f"(s1));
+}
+template <> NA_DEVICE void add_pair<__half>(float& d0, float& d1, float s0, float s1, uint32_t w) {
+  asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %2;\n add.rn.f32.f16 %0, lo, %3;\n add.rn.f32.f16 %1, hi, %4;\n}"
+      : "=f"(d0), "=f"(d1)
+      : "r"(w), "f"(s0), "f"(s1));
+}
+NA_DEVICE uint32_t bits16(__nv_bfloat16 x) { return __bfloat16_as_ushort(x); }
+NA_DEVICE uint32_t bits16(__half x) { return __half_as_ushort(x); }
+template <typename T> NA_DEVICE T neg_inf();
+template <> NA_DEVICE __nv_bfloat16 neg_inf() { return __ushort_as_bfloat16((unsigned short)0xff80u); }
+template <> NA_DEVICE __half neg_inf() { return __ushort_as_half((unsigned short)0xfc00u); }
+
 // Arrives on `bar` once for the whole warp, after every lane's earlier
 // memory operations: the barrier counts warps, not threads, which keeps
 // shared-memory atomics off the hot path.
@@ -319,14 +341,14 @@ struct Meeting {
 // union rows [u_r0, u_r1) and pieces [PB, PB+NU) of their windows, RB rows
 // at a time: each batch's tensor-memory loads are issued together and the RB
 // rows are independent streams of arithmetic.  Pass 1 writes
-// y = s log2e/sqrt(d) + table (bias log2e/sqrt(d), -inf outside the window)
-// back over S and takes the row maximum m; pass 2 writes P = exp2(y - m) as
+// y = s + table (the bias, -inf outside the window) back over S and takes
+// the row maximum m; pass 2 writes P = exp2((y - m) log2e/sqrt(d)) as
 // 16-bit pairs over S -- P row hr covers the S columns of row hr / 2, read by
 // an earlier or the same batch -- zeros outside the pieces, and returns the
 // sum of the rounded P.  Rows past u_r1 in the last batch repeat row u_r1-1:
 // they store the same values again and are left out of the sum.
 template <typename T, int KS, int D, int PB, int NU>
-NA_DEVICE float softmax_rows(uint32_t sbuf, const float* tl, int u_r0, int u_r1, int wr0, int er, float c) {
+NA_DEVICE float softmax_rows(uint32_t sbuf, const T* tl, int u_r0, int u_r1, int wr0, int er, float c) {
   using C = Cfg<KS, D>;
   constexpr int HW = C::HW, PW = HW / 2, NV = NU * 4, RB = 2;
   // start-column alignment of a piece window (row hr * HW + PB * 4) and of a P row (hr * PW)
@@ -346,20 +368,21 @@ NA_DEVICE float softmax_rows(uint32_t sbuf, const float* tl, int u_r0, int u_r1,
 #pragma unroll
     for (int j = 0; j < RB; ++j) {
       const int hr = min(r0 + j, last);
-      const float* tr = tl + ((unsigned)(hr - wr0) < (unsigned)KS ? hr + er : 2 * KS - 1) * C::TBL_W + PB * 4;
+      const T* tr = tl + ((unsigned)(hr - wr0) < (unsigned)KS ? hr + er : 2 * KS - 1) * C::TBL_W + PB * 4;
 #pragma unroll
       for (int e = 0; e < NV; e += 4) {
-        float2 b01, b23;
-        if constexpr (C::TBL_COPIES == 2) {
-          b01 = reinterpret_cast<const float2*>(tr)[e / 2];
-          b23 = reinterpret_cast<const float2*>(tr)[e / 2 + 1];
+        uint32_t b01, b23;  // entries e, e+1 and e+2, e+3
+        if constexpr (C::TBL_COPIES == 4) {
+          const uint2 w = *reinterpret_cast<const uint2*>(tr + e);
+          b01 = w.x;
+          b23 = w.y;
         } else {
-          b01 = make_float2(tr[e], tr[e + 1]);
-          b23 = make_float2(tr[e + 2], tr[e + 3]);
+          b01 = *reinterpret_cast<const uint32_t*>(tr + e);
+          b23 = *reinterpret_cast<const uint32_t*>(tr + e + 2);
         }
         float y0, y1, y2, y3;
-        fma2(y0, y1, __uint_as_float(v[j][e]), __uint_as_float(v[j][e + 1]), c, c, b01.x, b01.y);
-        fma2(y2, y3, __uint_as_float(v[j][e + 2]), __uint_as_float(v[j][e + 3]), c, c, b23.x, b23.y);
+        add_pair<T>(y0, y1, __uint_as_float(v[j][e]), __uint_as_float(v[j][e + 1]), b01);
+        add_pair<T>(y2, y3, __uint_as_float(v[j][e + 2]), __uint_as_float(v[j][e + 3]), b23);
         mx[j] = max3(mx[j], max3(y0, y1, y2), y3);
         v[j][e] = __float_as_uint(y0);
         v[j][e + 1] = __float_as_uint(y1);
@@ -373,6 +396,7 @@ NA_DEVICE float softmax_rows(uint32_t sbuf, const float* tl, int u_r0, int u_r1,
   float m = mx[0];
 #pragma unroll
   for (int j = 1; j < RB; ++j) m = fmaxf(m, mx[j]);
+  const float cm = -c * m;
 
   uint32_t z[PW];
 #pragma unroll
@@ -396,8 +420,8 @@ NA_DEVICE float softmax_rows(uint32_t sbuf, const float* tl, int u_r0, int u_r1,
 #pragma unroll
       for (int e = 0; e < NV; e += 4) {
         float a0, a1, a2, a3;
-        add2(a0, a1, __uint_as_float(v[j][e]), __uint_as_float(v[j][e + 1]), -m, -m);
-        add2(a2, a3, __uint_as_float(v[j][e + 2]), __uint_as_float(v[j][e + 3]), -m, -m);
+        fma2(a0, a1, __uint_as_float(v[j][e]), __uint_as_float(v[j][e + 1]), c, c, cm, cm);
+        fma2(a2, a3, __uint_as_float(v[j][e + 2]), __uint_as_float(v[j][e + 3]), c, c, cm, cm);
         const uint32_t pa = exp2_pair<T>(a0, a1), pb = exp2_pair<T>(a2, a3);
         acc_pair<T>(s0, s1, pa);
         acc_pair<T>(s0, s1, pb);
@@ -417,7 +441,7 @@ NA_DEVICE float softmax_rows(uint32_t sbuf, const float* tl, int u_r0, int u_r1,
 // window union, fixed at compile time, or over whole rows when the union is
 // wider (patches at the map border).
 template <typename T, int KS, int D, int PB = 0>
-NA_DEVICE float softmax_dispatch(int pb, int pe, uint32_t sbuf, const float* tl, int u_r0, int u_r1, int wr0,
+NA_DEVICE float softmax_dispatch(int pb, int pe, uint32_t sbuf, const T* tl, int u_r0, int u_r1, int wr0,
                                  int er, float c) {
   using C = Cfg<KS, D>;
   if constexpr (PB + C::NPU <= C::NPC) {
@@ -440,8 +464,8 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
-  float* tables = reinterpret_cast<float*>(smem + ST * C::STAGE_BYTES);
-  float* raws = reinterpret_cast<float*>(smem + ST * C::STAGE_BYTES + NB * C::TBL_BYTES);
+  T* tables = reinterpret_cast<T*>(smem + ST * C::STAGE_BYTES);
+  T* raws = reinterpret_cast<T*>(smem + ST * C::STAGE_BYTES + NB * C::TBL_BYTES);
   float* lsums = reinterpret_cast<float*>(smem + ST * C::STAGE_BYTES + NB * (C::TBL_BYTES + C::RAW_BYTES));
   uint64_t* bars =
       reinterpret_cast<uint64_t*>(smem + ST * C::STAGE_BYTES + NB * (C::TBL_BYTES + C::RAW_BYTES + C::LSUM_BYTES));
@@ -623,8 +647,8 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int pc0 = (wq & 1) * PQ + (l16 & 3);    // query column inside the tile
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
     const uint32_t sbuf = tmem + lane_base + C::s_col(g);
-    float* tbl = tables + g * (C::TBL_BYTES / 4);
-    float* raw = raws + g * (C::RAW_BYTES / 4);
+    T* tbl = tables + g * (C::TBL_BYTES / 2);
+    T* raw = raws + g * (C::RAW_BYTES / 2);
     const float c = p.scale_log2;
     const T* rpb = static_cast<const T*>(p.rpb);
     Meeting tmeet{bar_tbl(g), 0u, abort_flag, p.status};
@@ -633,34 +657,46 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     for (int t = blockIdx.x + g * gridDim.x; t < p.total; t += NB * gridDim.x, ++use) {
       const Pair pr = decode_pair<KS>(t, p);
       if (pr.h != cur_h) {
-        // New head: stage its bias (times log2e / sqrt(d)) with all loads in
-        // flight at once, then expand it into the group's table.
+        // New head: stage its bias with all loads in flight at once, then
+        // expand it into every copy of the group's table.
         constexpr int span = 2 * KS - 1;
         constexpr int PER = (C::RAW + 127) / 128;
-        float rv[PER];
+        T rv[PER];
 #pragma unroll
         for (int m = 0; m < PER; ++m) {
           const int idx = gtid + 128 * m;
-          rv[m] = (idx < C::RAW && rpb) ? to_f(rpb[(size_t)pr.h * C::RAW + idx]) * c : 0.f;
+          rv[m] = (idx < C::RAW && rpb) ? rpb[(size_t)pr.h * C::RAW + idx] : T(0.f);
         }
 #pragma unroll
         for (int m = 0; m < PER; ++m)
           if (gtid + 128 * m < C::RAW) raw[gtid + 128 * m] = rv[m];
         if (!tmeet.sync()) break;  // raw is visible; the previous pair's table reads are done
-        // one table column per thread; entry x of the second copy is entry x + 1 of the first
+        // copy 0, one table column per thread
         for (int col = gtid; col < C::TBL_W; col += 128) {
           const int blk = col / (KS + C::PAD), off = col % (KS + C::PAD);
           const bool live = blk < KS && off >= C::PAD;
           const int bc = blk + (off - C::PAD);
 #pragma unroll
-          for (int row = 0; row < C::TBL_ROWS; ++row) {
-            const float v = (live && row < span) ? raw[row * span + bc] : -INFINITY;
-            const int x = row * C::TBL_W + col;
-            tbl[x] = v;
-            if (C::TBL_COPIES == 2 && x > 0) tbl[C::TBL_N + x - 1] = v;
+          for (int row = 0; row < C::TBL_ROWS; ++row)
+            tbl[row * C::TBL_W + col] = (live && row < span) ? raw[row * span + bc] : neg_inf<T>();
+        }
+        if (!tmeet.sync()) break;  // copy 0 is complete
+        // copies 1..: entry y of copy q is entry y + q of copy 0 (-inf past
+        // its end), four entries per 8-byte store, shifted out of two
+        // aligned 8-byte loads of copy 0
+        {
+          constexpr int QUADS = C::TBL_N / 4;
+          const uint32_t ninf2 = bits16(neg_inf<T>()) * 0x10001u;
+          for (int u = gtid; u < (C::TBL_COPIES - 1) * QUADS; u += 128) {
+            const int q = 1 + u / QUADS, y = (u - (q - 1) * QUADS) * 4;
+            const uint2 lo = *reinterpret_cast<const uint2*>(tbl + y);
+            const uint2 hi = y + 4 < C::TBL_N ? *reinterpret_cast<const uint2*>(tbl + y + 4) : make_uint2(ninf2, ninf2);
+            const uint32_t w[4] = {lo.x, lo.y, hi.x, hi.y};
+            const int k = q >> 1, sh = (q & 1) * 16;
+            *reinterpret_cast<uint2*>(tbl + C::tbl_base(q) + y) =
+                make_uint2(__funnelshift_r(w[k], w[k + 1], sh), __funnelshift_r(w[k + 1], w[k + 2], sh));
           }
         }
-        if (C::TBL_COPIES == 2 && gtid == 0) tbl[2 * C::TBL_N - 1] = -INFINITY;
         if (!tmeet.sync()) break;
         cur_h = pr.h;
       }
@@ -678,8 +714,9 @@ na2d_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
       if (!mbar_wait(bar_s_full(g), use & 1, abort_flag, p.status)) break;
       tc_fence_after();
-      // this lane's table origin, in the copy where its pairs are 8-byte aligned
-      const float* tl = (C::TBL_COPIES == 2 && (colbase & 1)) ? tbl + C::TBL_N + colbase - 1 : tbl + colbase;
+      // this lane's table origin, in the copy where its entries are aligned
+      const int cq = colbase & (C::TBL_COPIES - 1);
+      const T* tl = tbl + C::tbl_base(cq) + colbase - cq;
       const float l = softmax_dispatch<T, KS, D>(pb, pe, sbuf, tl, u_r0, u_r1, wr0, er, c);
       // the row sum goes to the epilogue warpgroup through shared memory
       lsums[(g * 2 + (use & 1)) * 128 + wq * 32 + lane] = l;
