@@ -5,23 +5,28 @@
 // staged in shared memory -- re-planned for TMA, tcgen05 and tensor memory.
 //
 // Work unit: a "pair" of 8x8 query tiles stacked vertically (16 x 8
-// queries).  Each tile is one M = 64 MMA; tile A writes tensor-memory lanes
-// 0-15 of every 32-lane quarter, tile B lanes 16-31, so the two share the
-// same columns.  The pair's K and V halo -- (16+k-1) rows x (8+k-1, rounded
-// up to 8) columns -- is one TMA box each; tile B's halo starts 8 rows
-// further down inside the same buffer.
+// queries), one M = 128 MMA: tile A's queries are tensor-memory lanes 0-15
+// of every 32-lane quarter, tile B's lanes 16-31.  The query operand is
+// block-structured (tile A's queries in K block 0, tile B's in K block 1),
+// so each tile's S row is taken against its own halo: the pair's K and V
+// halo -- (16+k-1) rows x (8+k-1, rounded up to 8) columns -- is one TMA
+// box each, and tile B's halo starts rB rows further down inside the same
+// buffer.  Two single tiles of a map's last tile row share a pair that way.
 //
 // Roles of one persistent CTA per SM:
-//   warp 0      TMA producer (query patches, K halo, V halo; STAGES buffers)
-//   warp 1      tensor-memory allocation; one lane issues every tcgen05.mma
-//   warps 2..   NBUF softmax warpgroups; group g owns tensor-memory buffer g
-//               and every NBUF-th pair, so one group's P.V and epilogue
-//               overlap the other group's softmax.
+//   warp 0          TMA producer of the Q/K ring (query tiles, K halo)
+//   warp 3          TMA producer of the V ring
+//   warps 1..NBUF   one MMA issuer each, for its own tensor-memory buffer
+//                   (warp 1 also allocates and frees tensor memory)
+//   warpgroups 1..NBUF  softmax groups: group g owns buffer g and every
+//                   NBUF-th pair of the CTA
+//   last warpgroup  the epilogue of every pair, in order
 // Per pair:  S = Q K_halo^T (fp32, tensor memory) -> each softmax warp reads
 // the union of the windows of its two 4x4 patches (one per tile), adds the
-// bias and the -inf mask from a per-head table, keeps x = s + bias in place,
-// takes the row maximum, then writes P = exp2((x - max) log2e / sqrt(d)) in
-// 16 bits over S (zeros outside the union) -> O = P V_halo -> O / rowsum.
+// bias and the -inf mask from a per-head 16-bit table, keeps x = s + bias in
+// place, takes the row maximum, then writes P = exp2((x - max) log2e /
+// sqrt(d)) in 16 bits over S (zeros outside the union) -> O = P V_halo, in
+// the dead columns of S -> O / rowsum, rounded, stored by the epilogue.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
