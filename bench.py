@@ -78,18 +78,53 @@ def file_sha(path):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
+def strip_c_comments(text):
+    """C/C++ source without comments and without blank or repeated whitespace:
+    what the compiler sees, so an edit of comments alone keeps its hash."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    lines = ("".join(out)).splitlines()
+    return "\n".join(" ".join(ln.split()) for ln in lines if ln.strip())
+
+
+def code_sha(path):
+    """Hash of a kernel source with its comments stripped (see strip_c_comments)."""
+    with open(path) as f:
+        return hashlib.sha256(strip_c_comments(f.read()).encode()).hexdigest()[:16]
+
+
 def profiled_traffic(kernel_source, workload):
     """DRAM bytes per launch from the committed ncu summary of this kernel and
-    workload, if it was taken on the current source; else None."""
+    workload, if it was captured on code identical (comments aside) to the
+    current source; else None.  A summary records the hash of the file it
+    was captured on (source_sha256_16) and of its comment-free code
+    (code_sha256_16); only the latter is compared."""
     name = os.path.splitext(os.path.basename(kernel_source))[0]
     path = os.path.join(ROOT, "profiles", f"{name}_{workload}.md")
     try:
         text = open(path).read()
     except OSError:
         return None
-    sha = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
+    sha = re.search(r"code_sha256_16:\s*([0-9a-f]+)", text)
     tr = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not sha or not tr or sha.group(1) != file_sha(kernel_source):
+    if not sha or not tr or sha.group(1) != code_sha(kernel_source):
         return None
     return float(tr.group(1))
 
@@ -134,7 +169,10 @@ class ClockSampler:
             out, _ = self.proc.communicate()
         self.lines = [ln for ln in out.splitlines() if ln.strip()]
 
-    def summary(self):
+    def summary(self, window=None):
+        """Median SM clock, max clock and active throttle reasons of the samples
+        inside `window` (host time (t0, t1); default: the marked window)."""
+        window = window or self.window
         rows = []
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
@@ -147,7 +185,7 @@ class ClockSampler:
                 continue
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        inside = [r for r in rows if self.window and self.window[0] - 0.25 <= r[0] <= self.window[1] + 0.25]
+        inside = [r for r in rows if window and window[0] - 0.25 <= r[0] <= window[1] + 0.25]
         use, where = (inside, "timed region") if inside else (rows, "whole run (timed region shorter than a sample)")
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
         reasons = sorted({n for r in use for n, a in zip(names, r[3]) if a.lower() == "active"})
@@ -155,12 +193,24 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(use), "window": where}
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 # ------------------------------------------------------------- CPU oracle
 
-def cpu_oracle_throughput(w, seconds, rows_per_call=None):
-    """Times the fp64 oracle (all host threads) on a bounded sample of the
-    workload: passes over all (b, h) maps, or over as many as one pass of
-    about `seconds` allows, repeated until `seconds` have passed."""
+def cpu_oracle_throughput(w, seconds):
+    """Times the fp64 oracle on a bounded sample of the workload: with all
+    host threads, passes over all (b, h) maps, or over as many as one pass of
+    about `seconds` allows, repeated until `seconds` have passed; then with
+    one thread on one map for about a tenth of that."""
     import oracle
     from vision_sliding_window_b200.inputs import workload_inputs
 
@@ -169,8 +219,7 @@ def cpu_oracle_throughput(w, seconds, rows_per_call=None):
     rpb = rpb.double().numpy()
     nthreads = oracle.max_threads()
     maps = w.B * w.heads
-    # warm the thread pool on one map, then size the sample: whole passes over
-    # the workload (or over as many maps as fit), repeated until `seconds`
+    # warm the thread pool on one map, then size the sample
     oracle.forward_rows(q, k, v, rpb, w.ks, 0, w.H, nthreads)
     t0 = time.perf_counter()
     oracle.forward_rows(q, k, v, rpb, w.ks, 0, w.H, nthreads)
@@ -187,7 +236,19 @@ def cpu_oracle_throughput(w, seconds, rows_per_call=None):
     qn = passes * n_maps * w.H * w.W * w.ks * w.ks
     sample = (f"{passes} pass(es) over {n_maps} of {maps} (b, h) maps of {w.name} "
               f"({qn / 1e6:.2f} M query-neighbours, {dt:.1f} s)")
-    return {"value": qn / dt / 1e9, "unit": UNIT, "cores": nthreads, "kind": "oracle", "sample": sample}
+    # one thread: whole maps until a tenth of the budget has passed
+    rows1, t1 = 0, time.perf_counter()
+    while True:
+        oracle.forward_rows(q, k, v, rpb, w.ks, 0, w.H, 1)
+        rows1 += w.H
+        if time.perf_counter() - t1 >= seconds / 10:
+            break
+    dt1 = time.perf_counter() - t1
+    qn1 = rows1 * w.W * w.ks * w.ks
+    return {"value": qn / dt / 1e9, "unit": UNIT, "cores": nthreads, "kind": "oracle", "sample": sample,
+            "cpu_model": cpu_model(),
+            "one_thread": {"value": qn1 / dt1 / 1e9, "unit": UNIT,
+                           "sample": f"{rows1 // w.H} map(s) of {w.name}, {dt1:.1f} s"}}
 
 
 def run_reference(args, rank):
@@ -224,7 +285,8 @@ def run_reference(args, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(w, args.gpus),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle", "sample": sample,
+                         "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -246,6 +308,113 @@ def workload_config(w, n_gpus, extra=None):
 
 # -------------------------------------------------------------------- ours
 
+# The headline workloads besides stage1 that the line reports, each timed in
+# the same run (nested under "targets").
+TARGETS = ("hires_k7", "hires_k13")
+TARGET_STEPS = 400
+
+
+class Timer:
+    """Back-to-back na2d_forward launches of one workload, replayed from CUDA
+    graphs over R rotating input/output sets (R sets >= 3x L2)."""
+
+    def __init__(self, w, dev, rank, graph_steps):
+        import torch
+        from dataclasses import replace
+
+        from vision_sliding_window_b200 import na2d
+        from vision_sliding_window_b200.inputs import workload_inputs
+
+        self.w, self.dev, self.na2d = w, dev, na2d
+        # rank r holds batch entries [r*B, (r+1)*B) of the global batch (its own seed)
+        self.host = workload_inputs(replace(w, seed=w.seed + rank))
+        self.set_bytes = w.io_bytes
+        self.l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.R = max(2, math.ceil(3 * self.l2 / self.set_bytes))
+        self.sets = []
+        for _ in range(self.R):
+            q, k, v, rpb = (t.to(dev) for t in self.host)
+            self.sets.append((q, k, v, rpb, torch.empty_like(q)))
+        self.graph_steps = graph_steps
+        self.kind = na2d.forward_kernel(*w.shape(), w.ks, self.host[0].dtype)
+
+    def step(self, i):
+        q, k, v, rpb, out = self.sets[i % self.R]
+        self.na2d.forward(q, k, v, rpb, self.w.ks, out=out)
+
+    def warm(self, n):
+        import torch
+
+        for i in range(max(n, 0)):
+            self.step(i)
+        torch.cuda.synchronize(self.dev)
+        if self.na2d.device_status() != self.na2d.NA_OK:
+            raise SystemExit(f"device status not OK after warm-up of {self.w.name}")
+
+    def timed(self, steps, barrier=None):
+        """Device time (ms) of exactly `steps` launches, and the host window."""
+        import torch
+
+        G = max(1, min(self.graph_steps, steps))
+        n_full, rem = divmod(steps, G)
+
+        def capture(n):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for i in range(n):
+                    self.step(i)
+            return g
+
+        g_full = capture(G) if n_full else None
+        g_rem = capture(rem) if rem else None
+        if g_full is not None:
+            g_full.replay()  # one untimed replay of the captured graph
+        torch.cuda.synchronize(self.dev)
+        stream = torch.cuda.current_stream(self.dev)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if barrier:
+            barrier(self.dev)
+        torch.cuda.synchronize(self.dev)
+        t0 = time.time()
+        ev0.record(stream)
+        for _ in range(n_full):
+            g_full.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize(self.dev)
+        t1 = time.time()
+        if barrier:
+            barrier(self.dev)
+        status = self.na2d.device_status()
+        if status != self.na2d.NA_OK:
+            raise SystemExit(f"device status {self.na2d.status_str(status)} after timing {self.w.name}")
+        del g_full, g_rem
+        return ev0.elapsed_time(ev1), (t0, t1), G
+
+    def release(self):
+        self.sets = []
+
+
+def roofline_of(w, launch_s, kernel_kind, peaks, peak_src):
+    kernel_source = TC_SOURCE if kernel_kind == 1 else SIMT_SOURCE
+    kernel_name = "na2d_fwd_tc" if kernel_kind == 1 else "na2d_fwd_simt"
+    achieved_gbs = w.io_bytes / launch_s / 1e9
+    tflops = w.flops / launch_s / 1e12
+    return {
+        "bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        "frac": achieved_gbs / peaks["hbm_gbs"],
+        "traffic": profiled_traffic(kernel_source, w.name),
+        "traffic_kind": ("ncu dram__bytes_read.sum + dram__bytes_write.sum per launch; the output's "
+                         "writes still held in L2 when the kernel ends are not counted, so this is "
+                         "in effect the DRAM read traffic"),
+        "kernel": kernel_name, "launch_us": launch_s * 1e6, "peak_source": peak_src,
+        "algorithmic_bytes": w.io_bytes,
+        "tensor_view": {"achieved_tflops": tflops, "peak_tflops": peaks["bf16_tflops"],
+                        "frac": tflops / peaks["bf16_tflops"]},
+    }
+
+
 def main(argv=None):
     args = parse_args(argv)
     from vision_sliding_window_b200.dist import barrier, env_rank, max_over_ranks
@@ -258,7 +427,7 @@ def main(argv=None):
     import torch.distributed as dist
 
     from vision_sliding_window_b200 import na2d
-    from vision_sliding_window_b200.inputs import WORKLOADS, workload_inputs
+    from vision_sliding_window_b200.inputs import WORKLOADS
 
     w = WORKLOADS[args.workload]
     if not torch.cuda.is_available():
@@ -267,83 +436,54 @@ def main(argv=None):
     dev = torch.device("cuda", local_rank)
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    lib = na2d.load_library()
-    kernel_kind = na2d.forward_kernel(*w.shape(), w.ks, {"bf16": torch.bfloat16, "f16": torch.float16,
-                                                         "f32": torch.float32}[w.dtype])
-    kernel_source = TC_SOURCE if kernel_kind == 1 else SIMT_SOURCE
-    kernel_name = "na2d_fwd_tc" if kernel_kind == 1 else "na2d_fwd_simt"
-
-    # inputs: rank r holds batch entries [r*B, (r+1)*B) of the global batch (its own seed)
-    from dataclasses import replace
-    wr = replace(w, seed=w.seed + rank)
-    host = workload_inputs(wr)
-    set_bytes = w.io_bytes
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    R = max(2, math.ceil(3 * l2 / set_bytes))
-    sets = []
-    for r in range(R):
-        q, k, v, rpb = (t.to(dev) for t in host)
-        sets.append((q, k, v, rpb, torch.empty_like(q)))
-
-    def step(i):
-        q, k, v, rpb, out = sets[i % R]
-        na2d.forward(q, k, v, rpb, w.ks, out=out)
-
-    stream = torch.cuda.current_stream(dev)
-    for i in range(max(args.warmup, 0)):
-        step(i)
-    torch.cuda.synchronize(dev)
-    if na2d.device_status() != na2d.NA_OK:
-        raise SystemExit("device status not OK after warm-up")
-
-    # graphs of G steps (+ one for the remainder) so launches are back to back
-    G = max(1, min(args.graph_steps, args.steps))
-    n_full, rem = divmod(args.steps, G)
-
-    def capture(n, offset):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for i in range(n):
-                step(offset + i)
-        return g
-
-    g_full = capture(G, 0) if n_full else None
-    g_rem = capture(rem, 0) if rem else None
-    if g_full is not None:
-        g_full.replay()  # one untimed replay of the captured graph
-    torch.cuda.synchronize(dev)
+    na2d.load_library()
+    peaks, peak_src = load_peaks()
 
     sampler = ClockSampler(local_rank) if rank == 0 else None
     if sampler:
         sampler.start()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(dev)
-    torch.cuda.synchronize(dev)
-    t_host0 = time.time()
-    ev0.record(stream)
-    for _ in range(n_full):
-        g_full.replay()
-    if g_rem is not None:
-        g_rem.replay()
-    ev1.record(stream)
-    torch.cuda.synchronize(dev)
-    t_host1 = time.time()
-    barrier(dev)
-    local_ms = ev0.elapsed_time(ev1)
+
+    main_timer = Timer(w, dev, rank, args.graph_steps)
+    main_timer.warm(args.warmup)
+    local_ms, window, G = main_timer.timed(args.steps, barrier)
     total_ms = max_over_ranks(local_ms, dev)
     if sampler:
-        sampler.mark(t_host0, t_host1)
-    status = na2d.device_status()
-    if status != na2d.NA_OK:
-        raise SystemExit(f"device status {na2d.status_str(status)} after the timed region")
+        sampler.mark(*window)
+    host = main_timer.host
+    R, set_bytes, l2 = main_timer.R, main_timer.set_bytes, main_timer.l2
+    kernel_kind = main_timer.kind
+    main_timer.release()
 
-    # end to end through the host-buffer entry point (pinned buffers, copies timed)
+    # the other headline workloads, each timed the same way (same ranks, same order)
+    targets = {}
+    if args.workload == "stage1":
+        for name in TARGETS:
+            tw = WORKLOADS[name]
+            t = Timer(tw, dev, rank, args.graph_steps)
+            t.warm(max(args.warmup, 3))
+            n = max(args.steps, TARGET_STEPS)
+            ms, win, _ = t.timed(n, barrier)
+            ms = max_over_ranks(ms, dev)
+            launch = ms * 1e-3 / n
+            rl = roofline_of(tw, launch, t.kind, peaks, peak_src)
+            targets[name] = {
+                "workload": workload_config(tw, world)["workload"],
+                "steps": n, "us_per_launch": launch * 1e6,
+                "value": world * n * tw.query_neighbours / (ms * 1e-3) / 1e9, "unit": UNIT,
+                "gbs": rl["achieved"], "frac": rl["frac"], "tflops": rl["tensor_view"]["achieved_tflops"],
+                "traffic": rl["traffic"], "kernel": rl["kernel"], "window": win,
+            }
+            t.release()
+
+    # end to end through the host-buffer entry point (pinned host buffers,
+    # every step's copies in and out inside the timed region)
     pin = [t.pin_memory() for t in host]
     out_host = torch.empty_like(host[0]).pin_memory()
     ws = torch.empty(na2d.host_workspace_bytes(*w.shape(), w.ks, host[0].dtype), dtype=torch.uint8, device=dev)
     for _ in range(3):
         na2d.forward_host(*pin, out_host, w.ks, ws)
     torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(dev)
     torch.cuda.synchronize(dev)
@@ -361,18 +501,6 @@ def main(argv=None):
     value = world * args.steps * qn_step / (total_ms * 1e-3) / 1e9
     e2e_value = world * args.e2e_steps * qn_step / (e2e_ms * 1e-3) / 1e9
     launch_s = local_ms * 1e-3 / args.steps
-    peaks, peak_src = load_peaks()
-    achieved_gbs = w.io_bytes / launch_s / 1e9
-    tflops = w.flops / launch_s / 1e12
-    traffic = profiled_traffic(kernel_source, w.name)
-    roofline = {
-        "bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-        "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": traffic,
-        "kernel": kernel_name, "launch_us": launch_s * 1e6, "peak_source": peak_src,
-        "algorithmic_bytes": w.io_bytes,
-        "tensor_view": {"achieved_tflops": tflops, "peak_tflops": peaks["bf16_tflops"],
-                        "frac": tflops / peaks["bf16_tflops"]},
-    }
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -381,7 +509,7 @@ def main(argv=None):
             "l2": f"rotating {R} input/output sets ({R * set_bytes / 1e6:.0f} MB, L2 {l2 / 1e6:.0f} MB)",
             "timing": f"CUDA graphs of {G} steps, CUDA events on the launching stream, max over ranks",
         }),
-        "roofline": roofline,
+        "roofline": roofline_of(w, launch_s, kernel_kind, peaks, peak_src),
         "e2e": {"value": e2e_value, "unit": UNIT,
                 "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host),
                 "d2h_bytes_per_step": host[0].numel() * host[0].element_size(),
@@ -390,10 +518,13 @@ def main(argv=None):
     }
     if rank == 0:
         line["clocks"] = sampler.summary() if sampler else None
+        if targets:
+            for tv in targets.values():
+                tv["clocks"] = sampler.summary(tv.pop("window")) if sampler else None
+            line["targets"] = targets
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_oracle_throughput(w, args.cpu_seconds)
         print(json.dumps(line), flush=True)
-    del g_full, g_rem
     if world > 1:
         dist.destroy_process_group()
     return 0

@@ -136,9 +136,11 @@ na_status na2d_forward_host(const void *q_host, const void *k_host, const void *
  * rejected with NA_ERR_UNSUPPORTED; otherwise arguments, errors and results
  * are those of na2d_forward_host.  The call allocates nothing.
  *
- * The first call on a device looks up the array's device address on that
- * device (it must be the current device); make that first call before any
- * stream capture.  All calls on a device share the one array: calls whose
+ * Every call looks up the array's device address on the current device (a
+ * host-side lookup in the CUDA runtime, so a device reset between calls is
+ * harmless).  The first call on a device may load the library's kernels on
+ * it; make that first call before any stream capture.  All calls on a
+ * device share the one array: calls whose
  * work overlaps on the GPU (different streams, or host threads) race and may
  * return wrong results.  Each call writes everything it reads from the
  * array, so the contents left by an earlier call do not matter.

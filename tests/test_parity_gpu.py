@@ -79,6 +79,46 @@ def test_forward_workload_sampled(name):
     assert_close(got, want, w.dtype, name)
 
 
+# Every (dtype, k, d) the tensor-core kernel is built for, compared in full
+# with the oracle on maps that give each CTA several work units: 4x2x72x72
+# has a last tile row of single tiles (packed two per unit) and 324 units on
+# a 148-SM grid; 3x2x75x70 has a ragged last pair row (75 = 4*16 + 11) and a
+# ragged last tile column (70 = 8*8 + 6).
+TC_BUILDS = [(dt, ks, d) for dt in ("f16", "bf16") for ks in (3, 5, 7, 9, 11, 13) for d in (32, 64)]
+
+
+@pytest.mark.parametrize("dtype,ks,d", TC_BUILDS)
+def test_every_tc_build_in_full(dtype, ks, d):
+    for (B, heads, H, W), seed in (((4, 2, 72, 72), 7), ((3, 2, 75, 70), 8)):
+        assert na2d.forward_kernel(B, heads, H, W, d, ks, DTYPES[dtype]) == 1
+        q, k, v, rpb = make_inputs(B, heads, H, W, d, ks, dtype, seed=seed + ks, rpb_std=0.5)
+        out = run_forward(*to_dev(q, k, v, rpb), ks)
+        assert_close(out, oracle.forward(q, k, v, rpb, ks), dtype, f"{dtype} k={ks} d={d} {H}x{W}")
+
+
+@pytest.mark.parametrize("name", LARGE)
+def test_forward_workload_first_and_last_map_in_full(name):
+    """The first and the last (b, h) map of each large workload, every element."""
+    w = WORKLOADS[name]
+    q, k, v, rpb = workload_inputs(w)
+    out = run_forward(*to_dev(q, k, v, rpb), w.ks).cpu()
+    maps = w.B * w.heads
+    for m in (0, maps - 1):
+        want = oracle.forward_rows(q, k, v, rpb, w.ks, m * w.H, (m + 1) * w.H)
+        b, h = divmod(m, w.heads)
+        assert_close(out[b, h], want[b, h], w.dtype, f"{name} map {m}")
+
+
+@pytest.mark.parametrize("dtype,scale", [("bf16", 4.0), ("f16", 4.0), ("bf16", 8.0)])
+def test_wide_logit_spread_in_full(dtype, scale):
+    """q scaled up so that the scaled logits A/sqrt(d) span tens: the regime
+    where a 16-bit exponent argument or a loose shift would cost accuracy."""
+    q, k, v, rpb = make_inputs(2, 2, 40, 36, 32, 7, dtype, seed=61, rpb_std=0.5)
+    q = (q.float() * scale).to(q.dtype)
+    out = run_forward(*to_dev(q, k, v, rpb), 7)
+    assert_close(out, oracle.forward(q, k, v, rpb, 7), dtype, f"q x {scale}")
+
+
 def test_k_equals_map_matches_dense_self_attention_on_gpu():
     """Stage-4 (H = W = k = 7): the output is plain self-attention with the full bias."""
     w = WORKLOADS["stage4"]

@@ -3,7 +3,6 @@
 // variant of the forward pass and the wait-timeout probe.
 #include <cmath>
 #include <cstdint>
-#include <mutex>
 
 #include "na2d_common.cuh"
 #include "na2d_internal.h"
@@ -17,25 +16,15 @@ namespace {
 // out; read and cleared by na2d_device_status().
 __device__ unsigned int g_status_word;
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-unsigned* g_status_ptr[kMaxDevices] = {};
-
-// Device address of the status word on the current device (looked up once
-// per device with that device current).
+// Device address of the status word on the current device.  Looked up on
+// every call (a host-side table lookup in the runtime): an address cached
+// across calls would go stale if the process reset the device or created a
+// new primary context, and the next kernel would write through it.
 cudaError_t status_ptr(unsigned** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_status_word);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_status_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_status_word);
-    if (e != cudaSuccess) return e;
-    g_status_ptr[dev] = static_cast<unsigned*>(p);
-  }
-  *out = g_status_ptr[dev];
+  *out = static_cast<unsigned*>(p);
   return cudaSuccess;
 }
 

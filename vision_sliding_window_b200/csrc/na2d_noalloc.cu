@@ -6,8 +6,6 @@
 // allocates nothing.  It adds a path; the existing ones are unchanged.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "na2d.h"
 
 #define NA_EXPORT extern "C" __attribute__((visibility("default")))
@@ -19,25 +17,15 @@ namespace {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[NA2D_NOALLOC_SCRATCH_BYTES];
 
 // In host code g_noalloc_scratch names a host-side stand-in, not device
-// memory: its device address is looked up once per device, with that device
-// current, and cached.
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_addr[kMaxDevices] = {};
-
+// memory.  Its device address is looked up with the device current on every
+// call: the lookup is a host-side table access in the runtime, and an
+// address cached across calls would go stale after a device reset or a new
+// primary context in the same process.
 cudaError_t scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_addr[dev] = p;
-  }
-  *out = g_addr[dev];
+  *out = p;
   return cudaSuccess;
 }
 
