@@ -11,6 +11,7 @@ from .na2d_oracle import (  # noqa: F401
     qk_rpb,
     softmax,
     av,
+    backward,
     window_start,
     max_threads,
 )

@@ -218,6 +218,91 @@ void na2d_oracle_forward_points(const double *q, const double *k, const double *
     }
 }
 
+/*
+ * Gradients of NA_k: the backward pass of Eqs. (2)-(4).  NATTEN computes
+ * "QK+B" and "AV" and the gradients of their backward passes (Qiita write-up,
+ * section "NATTEN"); the NAT paper, Sec. 3.2, makes the operator a PyTorch
+ * autograd function.  For a scalar loss L with dout = dL/d(out), the chain
+ * rule through out = sum_n P_n v_n, P = softmax(z), z = A / sqrt(d),
+ * A_n = q . k_n + B_n gives, per query (i, j) and window entry n:
+ *
+ *   dP_n   = dout . v_n
+ *   dz_n   = P_n (dP_n - sum_m P_m dP_m)          (softmax Jacobian)
+ *   dA_n   = dz_n / sqrt(d)
+ *   dq(i,j)       += sum_n dA_n k_n
+ *   dk(r_n, t_n)  += dA_n q(i,j)
+ *   dv(r_n, t_n)  += P_n dout(i,j)
+ *   drpb[h][r_n - i + ks - 1][t_n - j + ks - 1] += dA_n
+ *
+ * dout, dq, dk, dv are [B][heads][H][W][d]; drpb is [heads][2ks-1][2ks-1]
+ * and may be NULL (no bias gradient).  The (b, h) maps run in parallel; each
+ * map accumulates its own bias gradient, and those are summed over b in
+ * order at the end.
+ */
+void na2d_oracle_backward(const double *q, const double *k, const double *v, const double *rpb,
+                          const double *dout, double *dq, double *dk, double *dv, double *drpb,
+                          long B, long heads, long H, long W, long d, long ks, int nthreads)
+{
+    long span = 2 * ks - 1, nn = ks * ks, maps = B * heads;
+    size_t total = (size_t)maps * H * W * d;
+    double scale = 1.0 / sqrt((double)d);
+    double *dB = (double *)calloc((size_t)maps * span * span, sizeof(double));
+    for (size_t t = 0; t < total; t++) dq[t] = dk[t] = dv[t] = 0.0;
+#pragma omp parallel num_threads(threads_for(nthreads))
+    {
+        double *P = (double *)malloc(sizeof(double) * (size_t)nn);
+        double *dP = (double *)malloc(sizeof(double) * (size_t)nn);
+#pragma omp for schedule(dynamic)
+        for (long bh = 0; bh < maps; bh++) {
+            long b = bh / heads, h = bh % heads;
+            for (long i = 0; i < H; i++) {
+                for (long j = 0; j < W; j++) {
+                    long si = na2d_oracle_window_start(i, H, ks);
+                    long sj = na2d_oracle_window_start(j, W, ks);
+                    size_t qi = idx5(b, h, i, j, heads, H, W, d);
+                    logits_one(q, k, rpb, b, h, i, j, heads, H, W, d, ks, P);
+                    softmax_row(P, nn, scale);
+                    double pdp = 0.0;
+                    for (long a = 0; a < ks; a++) {
+                        for (long c = 0; c < ks; c++) {
+                            long n = a * ks + c;
+                            size_t ki = idx5(b, h, si + a, sj + c, heads, H, W, d);
+                            double s = 0.0;
+                            for (long x = 0; x < d; x++) s += dout[qi + x] * v[ki + x];
+                            dP[n] = s;
+                            pdp += P[n] * s;
+                        }
+                    }
+                    for (long a = 0; a < ks; a++) {
+                        for (long c = 0; c < ks; c++) {
+                            long n = a * ks + c;
+                            size_t ki = idx5(b, h, si + a, sj + c, heads, H, W, d);
+                            double dA = P[n] * (dP[n] - pdp) * scale;
+                            for (long x = 0; x < d; x++) {
+                                dq[qi + x] += dA * k[ki + x];
+                                dk[ki + x] += dA * q[qi + x];
+                                dv[ki + x] += P[n] * dout[qi + x];
+                            }
+                            dB[((size_t)bh * span + (si + a - i + ks - 1)) * span + (sj + c - j + ks - 1)] += dA;
+                        }
+                    }
+                }
+            }
+        }
+        free(P);
+        free(dP);
+    }
+    if (drpb) {
+        for (long h = 0; h < heads; h++)
+            for (long e = 0; e < span * span; e++) {
+                double s = 0.0;
+                for (long b = 0; b < B; b++) s += dB[((size_t)(b * heads + h)) * span * span + e];
+                drpb[(size_t)h * span * span + e] = s;
+            }
+    }
+    free(dB);
+}
+
 int na2d_oracle_max_threads(void)
 {
     return threads_for(0);

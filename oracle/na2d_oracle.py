@@ -54,6 +54,7 @@ def _load():
                 + [_L] * 6
                 + [ctypes.c_int]
             )
+            lib.na2d_oracle_backward.argtypes = [_D] * 9 + [_L] * 6 + [ctypes.c_int]
             lib.na2d_oracle_max_threads.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -73,7 +74,7 @@ class swapped_library:
         lib = ctypes.CDLL(self.path)
         for fn in ("na2d_oracle_window_start", "na2d_oracle_qk_rpb", "na2d_oracle_softmax",
                    "na2d_oracle_av", "na2d_oracle_forward", "na2d_oracle_forward_rows",
-                   "na2d_oracle_forward_points", "na2d_oracle_max_threads"):
+                   "na2d_oracle_forward_points", "na2d_oracle_backward", "na2d_oracle_max_threads"):
             src, dst = getattr(self._saved, fn), getattr(lib, fn)
             dst.argtypes, dst.restype = src.argtypes, src.restype
         with _lock:
@@ -203,3 +204,16 @@ def forward_points(q, k, v, rpb, ks: int, points, nthreads: int = 0):
         _ptr(out), _ptr(logits), _ptr(attn), B, heads, H, W, d, ks, nthreads,
     )
     return out, logits, attn
+
+
+def backward(q, k, v, rpb, dout, ks: int, nthreads: int = 0):
+    """Gradients of L = sum(dout * NA_k(q, k, v, rpb)) with respect to q, k,
+    v and rpb (the backward of Eqs. (2)-(4)).  Returns (dq, dk, dv, drpb);
+    drpb is None when rpb is None."""
+    q, k, v, rpb, dout = _f64(q), _f64(k), _f64(v), _f64(rpb), _f64(dout)
+    B, heads, H, W, d = _shape(q, ks)
+    dq, dk, dv = (np.empty_like(q) for _ in range(3))
+    drpb = None if rpb is None else np.empty_like(rpb)
+    _load().na2d_oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(rpb), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                                 _ptr(drpb), B, heads, H, W, d, ks, nthreads)
+    return dq, dk, dv, drpb

@@ -1,5 +1,6 @@
 """Each plausible slip planted in a copy of the oracle source must make at
-least one pin of tests/test_oracle_pins.py fail.  The copies are compiled on
+least one pin of tests/test_oracle_pins.py (forward) or
+tests/test_oracle_backward_pins.py (backward) fail.  The copies are compiled on
 the CPU into a temporary directory; the committed oracle is never changed."""
 import inspect
 
@@ -7,6 +8,7 @@ import pytest
 
 import oracle
 from oracle import na2d_oracle as ora
+from tests import test_oracle_backward_pins as bwd_pins
 from tests import test_oracle_pins as pins
 
 MUTATIONS = {
@@ -29,10 +31,27 @@ MUTATIONS = {
 }
 
 
-def _pin_cases():
+# Slips in the backward pass, each checked against the backward pins.
+BACKWARD_MUTATIONS = {
+    "softmax Jacobian without the row term": ("double dA = P[n] * (dP[n] - pdp) * scale;",
+                                               "double dA = P[n] * dP[n] * scale;"),
+    "logit gradient not divided by sqrt(d)": ("double dA = P[n] * (dP[n] - pdp) * scale;",
+                                              "double dA = P[n] * (dP[n] - pdp);"),
+    "dk takes the key instead of the query": ("dk[ki + x] += dA * q[qi + x];", "dk[ki + x] += dA * k[ki + x];"),
+    "dv weighted by dP instead of P": ("dv[ki + x] += P[n] * dout[qi + x];", "dv[ki + x] += dP[n] * dout[qi + x];"),
+    "dq scattered to the key": ("dq[qi + x] += dA * k[ki + x];", "dq[ki + x] += dA * k[ki + x];"),
+    "bias gradient at the transposed displacement": (
+        "(si + a - i + ks - 1)) * span + (sj + c - j + ks - 1)] += dA;",
+        "(sj + c - j + ks - 1)) * span + (si + a - i + ks - 1)] += dA;"),
+    "dP from the query's own value": ("for (long x = 0; x < d; x++) s += dout[qi + x] * v[ki + x];",
+                                      "for (long x = 0; x < d; x++) s += dout[qi + x] * v[qi + x];"),
+}
+
+
+def _pin_cases(module=pins):
     """(name, callable) for every pin, with parametrized pins at each of their cases."""
     cases = []
-    for name, fn in inspect.getmembers(pins, inspect.isfunction):
+    for name, fn in inspect.getmembers(module, inspect.isfunction):
         if not name.startswith("test_"):
             continue
         marks = getattr(fn, "pytestmark", [])
@@ -57,6 +76,22 @@ def test_planted_mistake_is_caught(mutation, tmp_path):
     failed = []
     with ora.swapped_library(lib):
         for name, fn, kwargs in _pin_cases():
+            try:
+                fn(**kwargs)
+            except Exception:  # an assertion, or an error a pin provokes
+                failed.append(name)
+    assert failed, f"no pin caught the planted mistake: {mutation}"
+
+
+@pytest.mark.parametrize("mutation", sorted(BACKWARD_MUTATIONS))
+def test_planted_backward_mistake_is_caught(mutation, tmp_path):
+    old, new = BACKWARD_MUTATIONS[mutation]
+    text = ora.source_text()
+    assert text.count(old) == 1, f"mutation anchor not found once: {mutation}"
+    lib = ora.compile_variant(text.replace(old, new), str(tmp_path / "mutant.so"))
+    failed = []
+    with ora.swapped_library(lib):
+        for name, fn, kwargs in _pin_cases(bwd_pins):
             try:
                 fn(**kwargs)
             except Exception:  # an assertion, or an error a pin provokes
