@@ -106,10 +106,43 @@ na_status na2d_forward(const void *q, const void *k, const void *v, const void *
                        na_dtype dt, void *stream);
 
 /*
+ * Backward of na2d_forward: the gradients of a scalar loss L with respect to
+ * q, k, v and the bias table, given dout = dL/d(out).  NATTEN provides these
+ * for its "QK+B" and "AV" steps (Qiita write-up, section "NATTEN"); the NAT
+ * paper, Sec. 3.2, makes the operator an autograd function.  With
+ * P = softmax(A / sqrt(d)) over each query's window (Eqs. (2)-(4)):
+ *
+ *   dP_n = dout . v_n,  dA_n = P_n (dP_n - sum_m P_m dP_m) / sqrt(d),
+ *   dq = sum_n dA_n k_n,  dk(key) and dv(key) = sums over the queries whose
+ *   window holds the key of dA q and P dout,  drpb[h][displacement] = sum of
+ *   dA over all queries and window entries at that displacement.
+ *
+ * dout, dq, dk, dv: [B][heads][H][W][d] of type dt; dq, dk, dv are written,
+ * not accumulated into.  drpb: float32 [heads][2*ks-1][2*ks-1], written; NULL
+ * skips the bias gradient (which is defined whether rpb is NULL or not: a
+ * NULL rpb is a zero bias).  workspace: a 16-byte aligned device buffer of
+ * at least na2d_backward_workspace_bytes() bytes that the caller owns; its
+ * contents on entry do not matter (it holds two float64 per query between
+ * the passes).  Accumulation is float64 for NA_F32 and float32 for the
+ * 16-bit types; results are rounded to dt (drpb to float32).  The logits are
+ * recomputed from q, k and rpb: nothing from the forward call is needed.
+ */
+size_t na2d_backward_workspace_bytes(int B, int heads, int H, int W, int d, int ksize, na_dtype dt);
+na_status na2d_backward(const void *q, const void *k, const void *v, const void *rpb, const void *dout,
+                        void *dq, void *dk, void *dv, float *drpb, void *workspace, size_t workspace_bytes,
+                        int B, int heads, int H, int W, int d, int ksize, na_dtype dt, void *stream);
+
+/*
  * na2d_forward from HOST buffers: copies q, k, v (and rpb when not NULL)
  * host-to-device into the caller's device workspace, runs na2d_forward and
- * copies the result back to out_host, all enqueued on `stream` (one
- * cudaMemcpyAsync per buffer).  Pinned host memory makes the copies
+ * copies the result back to out_host, one cudaMemcpyAsync per buffer and
+ * batch chunk.  With B >= 2 the batch is cut into up to four chunks of whole
+ * batch entries that run on two streams of the library's own, forked from
+ * and joined back to `stream` with events, so that one chunk's copies
+ * overlap another chunk's kernel; the call is still ordered on `stream` as
+ * one operation.  The library creates those two streams and their events on
+ * the first such call on a device and keeps them; make that first call
+ * before any stream capture.  Pinned host memory makes the copies
  * asynchronous; the host buffers must stay valid until the stream is
  * synchronised.  workspace must be a 256-byte aligned device buffer of at
  * least na2d_forward_host_workspace_bytes() bytes.
@@ -134,7 +167,8 @@ na_status na2d_forward_host(const void *q_host, const void *k_host, const void *
  * (64 MiB) on every device that loads the library, held until the process
  * exits.  Shapes whose na2d_forward_host_workspace_bytes() exceeds that are
  * rejected with NA_ERR_UNSUPPORTED; otherwise arguments, errors and results
- * are those of na2d_forward_host.  The call allocates nothing.
+ * are those of na2d_forward_host.  The call allocates nothing and creates
+ * nothing: every copy and the kernel run in order on `stream`.
  *
  * Every call looks up the array's device address on the current device (a
  * host-side lookup in the CUDA runtime, so a device reset between calls is

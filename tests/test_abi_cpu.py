@@ -126,3 +126,24 @@ def test_binding_fails_loudly_without_library(tmp_path):
             na2d.load_library(str(tmp_path / "nope.so"))
     finally:
         na2d._lib = saved
+
+
+def bwd(lib, q=FAKE, k=FAKE, v=FAKE, rpb=None, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, drpb=FAKE, ws=FAKE,
+        ws_bytes=1 << 30, B=1, heads=1, H=8, W=8, d=32, ks=3, dt=na2d.NA_BF16):
+    return lib.na2d_backward(q, k, v, rpb, dout, dq, dk, dv, drpb, ws, ws_bytes, B, heads, H, W, d, ks, dt, None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(ks=4), dict(ks=11), dict(d=48), dict(H=0), dict(dt=5), dict(q=None), dict(dout=None), dict(dq=None),
+    dict(dk=None), dict(dv=None), dict(ws=None), dict(q=FAKE + 8), dict(dv=FAKE + 2), dict(drpb=FAKE + 4),
+    dict(rpb=FAKE + 4), dict(ws=FAKE + 8), dict(ws_bytes=16 * 64 - 1),
+])
+def test_backward_rejects_bad_arguments(lib, kw):
+    assert bwd(lib, **kw) == na2d.NA_ERR_INVALID_ARG
+
+
+def test_backward_workspace_and_empty_batch(lib):
+    # two float64 per query
+    assert lib.na2d_backward_workspace_bytes(2, 3, 10, 12, 32, 5, na2d.NA_F16) == 16 * 2 * 3 * 10 * 12
+    assert lib.na2d_backward_workspace_bytes(2, 3, 10, 12, 32, 4, na2d.NA_F16) == 0
+    assert bwd(lib, B=0, q=None, dq=None, ws=None) == na2d.NA_OK

@@ -3,6 +3,7 @@
 // variant of the forward pass and the wait-timeout probe.
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "na2d_common.cuh"
 #include "na2d_internal.h"
@@ -162,6 +163,29 @@ NA_EXPORT na_status na2d_forward(const void* q, const void* k, const void* v, co
   return from_cuda(launch_forward_simt(q, k, v, rpb, out, s, dt, cs));
 }
 
+NA_EXPORT size_t na2d_backward_workspace_bytes(int B, int heads, int H, int W, int d, int ksize, na_dtype dt) {
+  Shape s;
+  if (check_dtype(dt) != NA_OK || check_shape(B, heads, H, W, d, ksize, true, &s) != NA_OK) return 0;
+  return backward_workspace_bytes(s);
+}
+
+NA_EXPORT na_status na2d_backward(const void* q, const void* k, const void* v, const void* rpb, const void* dout,
+                                  void* dq, void* dk, void* dv, float* drpb, void* workspace,
+                                  size_t workspace_bytes, int B, int heads, int H, int W, int d, int ksize,
+                                  na_dtype dt, void* stream) {
+  Shape s;
+  na_status st = check_dtype(dt);
+  if (st == NA_OK) st = check_shape(B, heads, H, W, d, ksize, true, &s);
+  if (st != NA_OK) return st;
+  if (s.queries() == 0) return NA_OK;
+  for (const void* ptr : {q, k, v, dout, (const void*)dq, (const void*)dk, (const void*)dv, (const void*)workspace})
+    if (!ptr || !aligned16(ptr)) return NA_ERR_INVALID_ARG;
+  if ((rpb && !aligned16(rpb)) || (drpb && !aligned16(drpb))) return NA_ERR_INVALID_ARG;
+  if (workspace_bytes < backward_workspace_bytes(s)) return NA_ERR_INVALID_ARG;
+  return from_cuda(launch_backward_simt(q, k, v, rpb, dout, dq, dk, dv, drpb, workspace, s, dt,
+                                        (cudaStream_t)stream));
+}
+
 namespace {
 struct HostLayout {
   size_t q, k, v, rpb, out, total, tensor_bytes, rpb_bytes;
@@ -191,10 +215,48 @@ NA_EXPORT size_t na2d_forward_host_workspace_bytes(int B, int heads, int H, int 
   return host_layout(s, dt).total;
 }
 
-NA_EXPORT na_status na2d_forward_host(const void* q_host, const void* k_host, const void* v_host,
-                                      const void* rpb_host, void* out_host, void* workspace,
-                                      size_t workspace_bytes, int B, int heads, int H, int W, int d,
-                                      int ksize, na_dtype dt, void* stream) {
+namespace {
+// Two streams per device on which na2d_forward_host runs batch chunks side
+// by side -- the copies of one chunk overlap the kernel of the other -- and
+// the events that fork them from, and join them back to, the caller's
+// stream.  Created by the first such call on the device and kept for the
+// life of the process; calls are enqueued one at a time (a host mutex), so
+// the shared events are never recorded by two calls at once.
+struct Lanes {
+  cudaStream_t s[2];
+  cudaEvent_t fork, join[2];
+  bool ready;
+};
+constexpr int kMaxDevices = 64;
+std::mutex g_lanes_mu;
+Lanes g_lanes[kMaxDevices];
+
+cudaError_t lanes_for_current_device(Lanes** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  Lanes& L = g_lanes[dev];
+  if (!L.ready) {
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) e = cudaStreamCreateWithFlags(&L.s[i], cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L.fork, cudaEventDisableTiming);
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&L.join[i], cudaEventDisableTiming);
+    if (e != cudaSuccess) return e;
+    L.ready = true;
+  }
+  *out = &L;
+  return cudaSuccess;
+}
+
+// The host-buffer forward.  serial: every copy and the kernel in order on
+// the caller's stream.  Otherwise the batch is cut into up to four chunks of
+// whole batch entries, chunk c going to lane c % 2: its inputs' host-to-device
+// copies, its forward and its output's device-to-host copy, so that one
+// chunk's copies overlap another's kernel and copies in the two directions
+// overlap each other.
+na_status forward_host_impl(const void* q_host, const void* k_host, const void* v_host, const void* rpb_host,
+                            void* out_host, void* workspace, size_t workspace_bytes, int B, int heads, int H,
+                            int W, int d, int ksize, na_dtype dt, void* stream, bool serial) {
   Shape s;
   na_status st = check_dtype(dt);
   if (st == NA_OK) st = check_shape(B, heads, H, W, d, ksize, true, &s);
@@ -206,17 +268,72 @@ NA_EXPORT na_status na2d_forward_host(const void* q_host, const void* k_host, co
   if (workspace_bytes < L.total) return NA_ERR_INVALID_ARG;
   cudaStream_t cs = (cudaStream_t)stream;
   char* ws = static_cast<char*>(workspace);
-  cudaError_t e = cudaMemcpyAsync(ws + L.q, q_host, L.tensor_bytes, cudaMemcpyHostToDevice, cs);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(ws + L.k, k_host, L.tensor_bytes, cudaMemcpyHostToDevice, cs);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(ws + L.v, v_host, L.tensor_bytes, cudaMemcpyHostToDevice, cs);
-  if (e == cudaSuccess && rpb_host)
-    e = cudaMemcpyAsync(ws + L.rpb, rpb_host, L.rpb_bytes, cudaMemcpyHostToDevice, cs);
+  const char* qh = static_cast<const char*>(q_host);
+  const char* kh = static_cast<const char*>(k_host);
+  const char* vh = static_cast<const char*>(v_host);
+  char* oh = static_cast<char*>(out_host);
+  cudaError_t e = cudaSuccess;
+  if (rpb_host) e = cudaMemcpyAsync(ws + L.rpb, rpb_host, L.rpb_bytes, cudaMemcpyHostToDevice, cs);
   if (e != cudaSuccess) return NA_ERR_CUDA;
-  st = na2d_forward(ws + L.q, ws + L.k, ws + L.v, rpb_host ? ws + L.rpb : nullptr, ws + L.out, B, heads,
-                    H, W, d, ksize, dt, stream);
-  if (st != NA_OK) return st;
-  return from_cuda(cudaMemcpyAsync(out_host, ws + L.out, L.tensor_bytes, cudaMemcpyDeviceToHost, cs));
+  const void* rpb_dev = rpb_host ? ws + L.rpb : nullptr;
+  const int chunks = serial ? 1 : (B < 4 ? B : 4);
+  if (chunks <= 1) {
+    e = cudaMemcpyAsync(ws + L.q, qh, L.tensor_bytes, cudaMemcpyHostToDevice, cs);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(ws + L.k, kh, L.tensor_bytes, cudaMemcpyHostToDevice, cs);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(ws + L.v, vh, L.tensor_bytes, cudaMemcpyHostToDevice, cs);
+    if (e != cudaSuccess) return NA_ERR_CUDA;
+    st = na2d_forward(ws + L.q, ws + L.k, ws + L.v, rpb_dev, ws + L.out, B, heads, H, W, d, ksize, dt, stream);
+    if (st != NA_OK) return st;
+    return from_cuda(cudaMemcpyAsync(oh, ws + L.out, L.tensor_bytes, cudaMemcpyDeviceToHost, cs));
+  }
+  std::lock_guard<std::mutex> lk(g_lanes_mu);
+  Lanes* ln = nullptr;
+  if (lanes_for_current_device(&ln) != cudaSuccess) return NA_ERR_CUDA;
+  e = cudaEventRecord(ln->fork, cs);
+  for (int i = 0; i < 2 && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(ln->s[i], ln->fork, 0);
+  if (e != cudaSuccess) return NA_ERR_CUDA;
+  const size_t per_b = L.tensor_bytes / (size_t)B;
+  for (int c = 0; c < chunks && st == NA_OK; ++c) {
+    const int b0 = (int)((long long)B * c / chunks), b1 = (int)((long long)B * (c + 1) / chunks);
+    const size_t off = per_b * (size_t)b0, bytes = per_b * (size_t)(b1 - b0);
+    cudaStream_t ls = ln->s[c & 1];
+    e = cudaMemcpyAsync(ws + L.q + off, qh + off, bytes, cudaMemcpyHostToDevice, ls);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(ws + L.k + off, kh + off, bytes, cudaMemcpyHostToDevice, ls);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(ws + L.v + off, vh + off, bytes, cudaMemcpyHostToDevice, ls);
+    if (e != cudaSuccess) {
+      st = NA_ERR_CUDA;
+      break;
+    }
+    st = na2d_forward(ws + L.q + off, ws + L.k + off, ws + L.v + off, rpb_dev, ws + L.out + off, b1 - b0, heads, H,
+                      W, d, ksize, dt, (void*)ls);
+    if (st == NA_OK && cudaMemcpyAsync(oh + off, ws + L.out + off, bytes, cudaMemcpyDeviceToHost, ls) != cudaSuccess)
+      st = NA_ERR_CUDA;
+  }
+  // the caller's stream waits for both lanes, also after a failed enqueue
+  for (int i = 0; i < 2; ++i)
+    if (cudaEventRecord(ln->join[i], ln->s[i]) != cudaSuccess || cudaStreamWaitEvent(cs, ln->join[i], 0) != cudaSuccess)
+      st = NA_ERR_CUDA;
+  return st;
 }
+}  // namespace
+
+NA_EXPORT na_status na2d_forward_host(const void* q_host, const void* k_host, const void* v_host,
+                                      const void* rpb_host, void* out_host, void* workspace,
+                                      size_t workspace_bytes, int B, int heads, int H, int W, int d,
+                                      int ksize, na_dtype dt, void* stream) {
+  return forward_host_impl(q_host, k_host, v_host, rpb_host, out_host, workspace, workspace_bytes, B, heads, H, W,
+                           d, ksize, dt, stream, false);
+}
+
+// For na2d_noalloc.cu: the same call with every step on the caller's stream.
+namespace na2d {
+na_status forward_host_serial(const void* q_host, const void* k_host, const void* v_host, const void* rpb_host,
+                              void* out_host, void* workspace, size_t workspace_bytes, int B, int heads, int H,
+                              int W, int d, int ksize, na_dtype dt, void* stream) {
+  return forward_host_impl(q_host, k_host, v_host, rpb_host, out_host, workspace, workspace_bytes, B, heads, H, W,
+                           d, ksize, dt, stream, true);
+}
+}  // namespace na2d
 
 NA_EXPORT na_status na2d_device_status(void* stream) {
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return NA_ERR_CUDA;

@@ -22,6 +22,19 @@ cudaError_t launch_softmax_simt(float* attn, long long rows, int ks, float scale
 cudaError_t launch_av_simt(const float* attn, const void* v, void* out, const Shape& s,
                            na_dtype dt, cudaStream_t st);
 
+// Backward (na2d_bwd.cu): every dtype and head size; the workspace holds
+// two float64 per query.
+size_t backward_workspace_bytes(const Shape& s);
+cudaError_t launch_backward_simt(const void* q, const void* k, const void* v, const void* rpb, const void* dout,
+                                 void* dq, void* dk, void* dv, float* drpb, void* workspace, const Shape& s,
+                                 na_dtype dt, cudaStream_t st);
+
+// na2d_forward_host with every copy and the kernel in order on the
+// caller's stream (na2d_api.cu); used by na2d_forward_host_noalloc.
+na_status forward_host_serial(const void* q_host, const void* k_host, const void* v_host, const void* rpb_host,
+                              void* out_host, void* workspace, size_t workspace_bytes, int B, int heads, int H,
+                              int W, int d, int ksize, na_dtype dt, void* stream);
+
 // Tensor-core fused forward (na2d_tc.cu), fp16/bf16.
 bool forward_tc_supported(const Shape& s, na_dtype dt);
 cudaError_t launch_forward_tc(const void* q, const void* k, const void* v, const void* rpb,

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include "na2d.h"
+#include "na2d_internal.h"
 
 #define NA_EXPORT extern "C" __attribute__((visibility("default")))
 
@@ -47,6 +48,6 @@ NA_EXPORT na_status na2d_forward_host_noalloc(const void* q_host, const void* k_
   if (need > NA2D_NOALLOC_SCRATCH_BYTES) return NA_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return NA_ERR_CUDA;
-  return na2d_forward_host(q_host, k_host, v_host, rpb_host, out_host, scratch, NA2D_NOALLOC_SCRATCH_BYTES, B,
-                           heads, H, W, d, ksize, dt, stream);
+  return na2d::forward_host_serial(q_host, k_host, v_host, rpb_host, out_host, scratch, NA2D_NOALLOC_SCRATCH_BYTES,
+                                   B, heads, H, W, d, ksize, dt, stream);
 }

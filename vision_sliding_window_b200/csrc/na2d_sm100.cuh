@@ -55,6 +55,16 @@ NA_DEVICE bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag
   }
 }
 
+// Waits, bounded but regardless of the abort flag, for a phase that work
+// already in flight will complete (TMA copies landing, MMAs finishing):
+// used after giving up, so that nothing still writes shared or tensor
+// memory when the CTA exits.
+NA_DEVICE void mbar_wait_settle(uint32_t bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+}
+
 // ------------------------------------------------------------------ TMA
 // 5-D tiled load of the box at coordinates (c0 innermost .. c4) into shared
 // memory, completing `bytes` of transaction count on `bar`.

@@ -25,6 +25,7 @@ EXPORTS = (
     "na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward",
     "na2d_forward_host_workspace_bytes", "na2d_forward_host", "na2d_forward_host_noalloc", "na2d_forward_kernel",
     "na2d_device_status", "na2d_debug_timeout_probe", "na_status_str",
+    "na2d_backward_workspace_bytes", "na2d_backward",
 )
 
 
@@ -59,13 +60,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.na2d_forward_host.argtypes = [vp, vp, vp, vp, vp, vp, sz, *shape, i, vp]
         lib.na2d_forward_host_noalloc.argtypes = [vp, vp, vp, vp, vp, *shape, i, vp]
         lib.na2d_forward_kernel.argtypes = [*shape, i]
+        lib.na2d_backward_workspace_bytes.argtypes = [*shape, i]
+        lib.na2d_backward_workspace_bytes.restype = sz
+        lib.na2d_backward.argtypes = [vp] * 10 + [sz, *shape, i, vp]
         lib.na2d_device_status.argtypes = [vp]
         lib.na2d_debug_timeout_probe.argtypes = [ctypes.c_uint, vp]
         lib.na_status_str.argtypes = [i]
         lib.na_status_str.restype = ctypes.c_char_p
         for name in ("na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward",
                      "na2d_forward_host", "na2d_forward_host_noalloc", "na2d_forward_kernel", "na2d_device_status",
-                     "na2d_debug_timeout_probe"):
+                     "na2d_debug_timeout_probe", "na2d_backward"):
             getattr(lib, name).restype = i
         _lib = lib
         return lib
@@ -155,6 +159,28 @@ def av(attn, v, ksize: int, out=None):
     _check(load_library().na2d_av(_ptr(attn), _ptr(v), _ptr(out), B, heads, H, W, d, ksize,
                                   _DT[v.dtype], _stream(v)), "na2d_av")
     return out
+
+
+def backward(q, k, v, rpb, dout, ksize: int, with_rpb_grad: bool = True, workspace=None):
+    """Gradients of a scalar loss through the NA forward (na2d_backward):
+    returns (dq, dk, dv, drpb), drpb float32 [heads, 2k-1, 2k-1] or None."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (dout, "dout")):
+        _need(t, n, q.dtype)
+    if rpb is not None:
+        _need(rpb, "rpb", q.dtype)
+    B, heads, H, W, d = _dims(q)
+    lib = load_library()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    drpb = (torch.empty((heads, 2 * ksize - 1, 2 * ksize - 1), device=q.device, dtype=torch.float32)
+            if with_rpb_grad else None)
+    need = int(lib.na2d_backward_workspace_bytes(B, heads, H, W, d, ksize, _DT[q.dtype]))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace")
+    _check(lib.na2d_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(rpb), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                             _ptr(drpb), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                             B, heads, H, W, d, ksize, _DT[q.dtype], _stream(q)), "na2d_backward")
+    return dq, dk, dv, drpb
 
 
 def host_workspace_bytes(B, heads, H, W, d, ksize, dtype) -> int:
