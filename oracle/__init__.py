@@ -12,6 +12,7 @@ from .na2d_oracle import (  # noqa: F401
     softmax,
     av,
     backward,
+    sasa_forward,
     window_start,
     max_threads,
 )

@@ -303,6 +303,63 @@ void na2d_oracle_backward(const double *q, const double *k, const double *v, con
     free(dB);
 }
 
+/*
+ * SASA (stand-alone self-attention): the centred k x k window of every
+ * query, with the positions outside the map taken as zero padding.  The NAT
+ * paper, Sec. 3.2, calls SASA a special case of NA on a zero-padded input;
+ * the Qiita write-up's SASA/NA drawing shows the difference at the borders
+ * (SASA's window stays centred and reaches into the padding, NA's is
+ * shifted inward).  Per query (i, j), window entry (a, c) is the position
+ * (i - ks/2 + a, j - ks/2 + c); there the key and value are the map's when
+ * the position is inside the map and zero otherwise, and the bias is the
+ * table's entry for that displacement (a - ks/2, c - ks/2) in both cases:
+ *
+ *   A_n = q . key_n + B[h][a][c],  out = sum_n softmax(A / sqrt(d))_n value_n.
+ */
+void na2d_oracle_sasa_forward(const double *q, const double *k, const double *v, const double *rpb,
+                              double *out, long B, long heads, long H, long W, long d, long ks,
+                              int nthreads)
+{
+    long rows = B * heads * H, span = 2 * ks - 1, nn = ks * ks, half = ks / 2;
+    double scale = 1.0 / sqrt((double)d);
+#pragma omp parallel num_threads(threads_for(nthreads))
+    {
+        double *A = (double *)malloc(sizeof(double) * (size_t)nn);
+#pragma omp for schedule(dynamic)
+        for (long row = 0; row < rows; row++) {
+            long i = row % H, bh = row / H, h = bh % heads, b = bh / heads;
+            for (long j = 0; j < W; j++) {
+                const double *qv = q + idx5(b, h, i, j, heads, H, W, d);
+                for (long a = 0; a < ks; a++) {
+                    for (long c = 0; c < ks; c++) {
+                        long r = i - half + a, t = j - half + c;
+                        double dot = 0.0;
+                        if (r >= 0 && r < H && t >= 0 && t < W) {
+                            const double *kv = k + idx5(b, h, r, t, heads, H, W, d);
+                            for (long x = 0; x < d; x++) dot += qv[x] * kv[x];
+                        }
+                        double bias = rpb ? rpb[((size_t)h * span + (a - half + ks - 1)) * span + (c - half + ks - 1)]
+                                          : 0.0;
+                        A[a * ks + c] = dot + bias;
+                    }
+                }
+                softmax_row(A, nn, scale);
+                double *o = out + idx5(b, h, i, j, heads, H, W, d);
+                for (long x = 0; x < d; x++) o[x] = 0.0;
+                for (long a = 0; a < ks; a++) {
+                    for (long c = 0; c < ks; c++) {
+                        long r = i - half + a, t = j - half + c;
+                        if (r < 0 || r >= H || t < 0 || t >= W) continue;  /* zero value */
+                        const double *vv = v + idx5(b, h, r, t, heads, H, W, d);
+                        for (long x = 0; x < d; x++) o[x] += A[a * ks + c] * vv[x];
+                    }
+                }
+            }
+        }
+        free(A);
+    }
+}
+
 int na2d_oracle_max_threads(void)
 {
     return threads_for(0);

@@ -55,6 +55,7 @@ def _load():
                 + [ctypes.c_int]
             )
             lib.na2d_oracle_backward.argtypes = [_D] * 9 + [_L] * 6 + [ctypes.c_int]
+            lib.na2d_oracle_sasa_forward.argtypes = [_D] * 5 + [_L] * 6 + [ctypes.c_int]
             lib.na2d_oracle_max_threads.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -74,7 +75,8 @@ class swapped_library:
         lib = ctypes.CDLL(self.path)
         for fn in ("na2d_oracle_window_start", "na2d_oracle_qk_rpb", "na2d_oracle_softmax",
                    "na2d_oracle_av", "na2d_oracle_forward", "na2d_oracle_forward_rows",
-                   "na2d_oracle_forward_points", "na2d_oracle_backward", "na2d_oracle_max_threads"):
+                   "na2d_oracle_forward_points", "na2d_oracle_backward", "na2d_oracle_sasa_forward",
+                   "na2d_oracle_max_threads"):
             src, dst = getattr(self._saved, fn), getattr(lib, fn)
             dst.argtypes, dst.restype = src.argtypes, src.restype
         with _lock:
@@ -217,3 +219,16 @@ def backward(q, k, v, rpb, dout, ks: int, nthreads: int = 0):
     _load().na2d_oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(rpb), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
                                  _ptr(drpb), B, heads, H, W, d, ks, nthreads)
     return dq, dk, dv, drpb
+
+
+def sasa_forward(q, k, v, rpb, ks: int, nthreads: int = 0) -> np.ndarray:
+    """SASA: the centred ks x ks window with zero keys and values outside the
+    map (NA on a zero-padded input, NAT Sec. 3.2): [B, heads, H, W, d]."""
+    q, k, v, rpb = _f64(q), _f64(k), _f64(v), _f64(rpb)
+    B, heads, H, W, d = q.shape
+    if ks % 2 != 1 or ks < 1:
+        raise ValueError(f"kernel size {ks} must be odd")
+    out = np.empty_like(q)
+    _load().na2d_oracle_sasa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(rpb), _ptr(out), B, heads, H, W, d, ks,
+                                     nthreads)
+    return out

@@ -1,6 +1,7 @@
 """Each plausible slip planted in a copy of the oracle source must make at
-least one pin of tests/test_oracle_pins.py (forward) or
-tests/test_oracle_backward_pins.py (backward) fail.  The copies are compiled on
+least one pin of tests/test_oracle_pins.py (forward),
+tests/test_oracle_backward_pins.py (backward) or tests/test_oracle_sasa_pins.py
+(SASA) fail.  The copies are compiled on
 the CPU into a temporary directory; the committed oracle is never changed."""
 import inspect
 
@@ -10,6 +11,7 @@ import oracle
 from oracle import na2d_oracle as ora
 from tests import test_oracle_backward_pins as bwd_pins
 from tests import test_oracle_pins as pins
+from tests import test_oracle_sasa_pins as sasa_pins
 
 MUTATIONS = {
     "bias dropped": ("A[a * ks + c] = dot + bias_at(rpb, h, ks, r - i, t - j);",
@@ -45,6 +47,18 @@ BACKWARD_MUTATIONS = {
         "(sj + c - j + ks - 1)) * span + (si + a - i + ks - 1)] += dA;"),
     "dP from the query's own value": ("for (long x = 0; x < d; x++) s += dout[qi + x] * v[ki + x];",
                                       "for (long x = 0; x < d; x++) s += dout[qi + x] * v[qi + x];"),
+}
+
+
+# Slips in SASA, each checked against the SASA pins.
+SASA_MUTATIONS = {
+    "window clamped like NA": ("long r = i - half + a, t = j - half + c;\n                        double dot = 0.0;",
+                               "long r = na2d_oracle_window_start(i, H, ks) + a, t = na2d_oracle_window_start(j, W, ks) + c;\n                        double dot = 0.0;"),
+    "padding left out of the softmax": ("                        A[a * ks + c] = dot + bias;",
+                                        "                        A[a * ks + c] = (r >= 0 && r < H && t >= 0 && t < W) ? dot + bias : -INFINITY;"),
+    "no bias on the padding": ("                        A[a * ks + c] = dot + bias;",
+                               "                        A[a * ks + c] = (r >= 0 && r < H && t >= 0 && t < W) ? dot + bias : 0.0;"),
+    "bias index off by one": ("(a - half + ks - 1)) * span + (c - half + ks - 1)]", "(a - half + ks)) * span + (c - half + ks - 2)]"),
 }
 
 
@@ -92,6 +106,22 @@ def test_planted_backward_mistake_is_caught(mutation, tmp_path):
     failed = []
     with ora.swapped_library(lib):
         for name, fn, kwargs in _pin_cases(bwd_pins):
+            try:
+                fn(**kwargs)
+            except Exception:  # an assertion, or an error a pin provokes
+                failed.append(name)
+    assert failed, f"no pin caught the planted mistake: {mutation}"
+
+
+@pytest.mark.parametrize("mutation", sorted(SASA_MUTATIONS))
+def test_planted_sasa_mistake_is_caught(mutation, tmp_path):
+    old, new = SASA_MUTATIONS[mutation]
+    text = ora.source_text()
+    assert text.count(old) == 1, f"mutation anchor not found once: {mutation}"
+    lib = ora.compile_variant(text.replace(old, new), str(tmp_path / "mutant.so"))
+    failed = []
+    with ora.swapped_library(lib):
+        for name, fn, kwargs in _pin_cases(sasa_pins):
             try:
                 fn(**kwargs)
             except Exception:  # an assertion, or an error a pin provokes
