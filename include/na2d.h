@@ -133,14 +133,35 @@ na_status na2d_backward(const void *q, const void *k, const void *v, const void 
                         int B, int heads, int H, int W, int d, int ksize, na_dtype dt, void *stream);
 
 /*
+ * SASA (stand-alone self-attention): every query attends to its CENTRED
+ * ks x ks window, positions outside the map being zero padding (zero key
+ * and value; the table's bias still applies at every window position).
+ * The NAT paper, Sec. 3.2, calls SASA NA on a zero-padded input, and the
+ * Qiita write-up's SASA/NA drawing shows the two windows at the borders;
+ * that is how this call computes it: q, k and v are padded by ks/2 zero
+ * pixels on every side into the workspace, na2d_forward runs on the padded
+ * map, and the original pixels' outputs are written to out.
+ *
+ * Layouts, dtypes, rpb and errors as na2d_forward, except that ksize may
+ * exceed H and W (odd, 1 .. 63).  workspace: a 256-byte aligned device
+ * buffer of at least na2d_sasa_workspace_bytes() bytes that the caller owns
+ * (the padded q, k, v and output); its contents on entry do not matter.
+ */
+size_t na2d_sasa_workspace_bytes(int B, int heads, int H, int W, int d, int ksize, na_dtype dt);
+na_status na2d_sasa_forward(const void *q, const void *k, const void *v, const void *rpb, void *out,
+                            void *workspace, size_t workspace_bytes,
+                            int B, int heads, int H, int W, int d, int ksize,
+                            na_dtype dt, void *stream);
+
+/*
  * na2d_forward from HOST buffers: copies q, k, v (and rpb when not NULL)
  * host-to-device into the caller's device workspace, runs na2d_forward and
  * copies the result back to out_host, one cudaMemcpyAsync per buffer and
  * batch chunk.  With B >= 2 the batch is cut into up to four chunks of whole
- * batch entries that run on two streams of the library's own, forked from
- * and joined back to `stream` with events, so that one chunk's copies
- * overlap another chunk's kernel; the call is still ordered on `stream` as
- * one operation.  The library creates those two streams and their events on
+ * batch entries, each on a stream of the library's own, forked from and
+ * joined back to `stream` with events, so that one chunk's copies overlap
+ * another chunk's kernel; the call is still ordered on `stream` as one
+ * operation.  The library creates those four streams and their events on
  * the first such call on a device and keeps them; make that first call
  * before any stream capture.  Pinned host memory makes the copies
  * asynchronous; the host buffers must stay valid until the stream is

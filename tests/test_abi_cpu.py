@@ -147,3 +147,16 @@ def test_backward_workspace_and_empty_batch(lib):
     assert lib.na2d_backward_workspace_bytes(2, 3, 10, 12, 32, 5, na2d.NA_F16) == 16 * 2 * 3 * 10 * 12
     assert lib.na2d_backward_workspace_bytes(2, 3, 10, 12, 32, 4, na2d.NA_F16) == 0
     assert bwd(lib, B=0, q=None, dq=None, ws=None) == na2d.NA_OK
+
+
+def test_sasa_arguments(lib):
+    # any odd k, even one larger than the map; workspace: padded q, k, v and output
+    need = lib.na2d_sasa_workspace_bytes(1, 1, 5, 6, 32, 7, na2d.NA_BF16)
+    assert need == 4 * ((1 * 1 * 11 * 12 * 32 * 2 + 255) // 256 * 256)
+    assert lib.na2d_sasa_workspace_bytes(1, 1, 5, 6, 32, 8, na2d.NA_BF16) == 0
+    args = (FAKE, FAKE, FAKE, None, FAKE)
+    assert lib.na2d_sasa_forward(*args, FAKE, need - 1, 1, 1, 5, 6, 32, 7, na2d.NA_BF16, None) == na2d.NA_ERR_INVALID_ARG
+    assert lib.na2d_sasa_forward(*args, FAKE + 16, need, 1, 1, 5, 6, 32, 7, na2d.NA_BF16, None) == na2d.NA_ERR_INVALID_ARG
+    assert lib.na2d_sasa_forward(None, FAKE, FAKE, None, FAKE, FAKE, need, 1, 1, 5, 6, 32, 7, na2d.NA_BF16,
+                                 None) == na2d.NA_ERR_INVALID_ARG
+    assert lib.na2d_sasa_forward(*args, None, 0, 0, 1, 5, 6, 32, 7, na2d.NA_BF16, None) == na2d.NA_OK

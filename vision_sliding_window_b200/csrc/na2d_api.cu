@@ -187,6 +187,49 @@ NA_EXPORT na_status na2d_backward(const void* q, const void* k, const void* v, c
 }
 
 namespace {
+// SASA takes any odd k: its padded map (H + k - 1 by W + k - 1) always holds
+// a window.
+na_status check_sasa_shape(int B, int heads, int H, int W, int d, int ks, Shape* s) {
+  if (B < 0 || heads < 0 || H < 1 || W < 1) return NA_ERR_INVALID_ARG;
+  if (ks < 1 || (ks & 1) == 0 || ks > 63) return NA_ERR_INVALID_ARG;
+  if (d != 16 && d != 32 && d != 64 && d != 128) return NA_ERR_INVALID_ARG;
+  const long double n = (long double)B * heads * (H + ks - 1) * (W + ks - 1);
+  if (n * (long double)(d > ks * ks ? d : ks * ks) >= (long double)(1ll << 62)) return NA_ERR_INVALID_ARG;
+  *s = Shape{B, heads, H, W, d, ks};
+  return NA_OK;
+}
+}  // namespace
+
+NA_EXPORT size_t na2d_sasa_workspace_bytes(int B, int heads, int H, int W, int d, int ksize, na_dtype dt) {
+  Shape s;
+  if (check_dtype(dt) != NA_OK || check_sasa_shape(B, heads, H, W, d, ksize, &s) != NA_OK) return 0;
+  return sasa_workspace_bytes(s, elem_size(dt));
+}
+
+NA_EXPORT na_status na2d_sasa_forward(const void* q, const void* k, const void* v, const void* rpb, void* out,
+                                      void* workspace, size_t workspace_bytes, int B, int heads, int H, int W,
+                                      int d, int ksize, na_dtype dt, void* stream) {
+  Shape s;
+  na_status st = check_dtype(dt);
+  if (st == NA_OK) st = check_sasa_shape(B, heads, H, W, d, ksize, &s);
+  if (st != NA_OK) return st;
+  if (s.queries() == 0) return NA_OK;
+  for (const void* ptr : {q, k, v, (const void*)out})
+    if (!ptr || !aligned16(ptr)) return NA_ERR_INVALID_ARG;
+  if (rpb && !aligned16(rpb)) return NA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NA_ERR_INVALID_ARG;
+  const size_t es = elem_size(dt);
+  if (workspace_bytes < sasa_workspace_bytes(s, es)) return NA_ERR_INVALID_ARG;
+  cudaStream_t cs = (cudaStream_t)stream;
+  void *qp, *kp, *vp, *outp;
+  if (launch_sasa_pad(q, k, v, workspace, s, es, cs, &qp, &kp, &vp, &outp) != cudaSuccess) return NA_ERR_CUDA;
+  const int pad = ksize / 2;
+  st = na2d_forward(qp, kp, vp, rpb, outp, B, heads, H + 2 * pad, W + 2 * pad, d, ksize, dt, stream);
+  if (st != NA_OK) return st;
+  return from_cuda(launch_sasa_crop(outp, out, s, es, cs));
+}
+
+namespace {
 struct HostLayout {
   size_t q, k, v, rpb, out, total, tensor_bytes, rpb_bytes;
 };
@@ -216,15 +259,18 @@ NA_EXPORT size_t na2d_forward_host_workspace_bytes(int B, int heads, int H, int 
 }
 
 namespace {
-// Two streams per device on which na2d_forward_host runs batch chunks side
-// by side -- the copies of one chunk overlap the kernel of the other -- and
-// the events that fork them from, and join them back to, the caller's
+// Streams per device on which na2d_forward_host runs batch chunks side by
+// side, one chunk per stream -- the host-to-device copies of one chunk
+// overlap the kernel and the device-to-host copy of the previous ones, and
+// no stream holds a chunk's input copy behind another chunk's output copy --
+// and the events that fork them from, and join them back to, the caller's
 // stream.  Created by the first such call on the device and kept for the
 // life of the process; calls are enqueued one at a time (a host mutex), so
 // the shared events are never recorded by two calls at once.
+constexpr int kLanes = 4;
 struct Lanes {
-  cudaStream_t s[2];
-  cudaEvent_t fork, join[2];
+  cudaStream_t s[kLanes];
+  cudaEvent_t fork, join[kLanes];
   bool ready;
 };
 constexpr int kMaxDevices = 64;
@@ -238,9 +284,10 @@ cudaError_t lanes_for_current_device(Lanes** out) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   Lanes& L = g_lanes[dev];
   if (!L.ready) {
-    for (int i = 0; i < 2 && e == cudaSuccess; ++i) e = cudaStreamCreateWithFlags(&L.s[i], cudaStreamNonBlocking);
+    for (int i = 0; i < kLanes && e == cudaSuccess; ++i) e = cudaStreamCreateWithFlags(&L.s[i], cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L.fork, cudaEventDisableTiming);
-    for (int i = 0; i < 2 && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&L.join[i], cudaEventDisableTiming);
+    for (int i = 0; i < kLanes && e == cudaSuccess; ++i)
+      e = cudaEventCreateWithFlags(&L.join[i], cudaEventDisableTiming);
     if (e != cudaSuccess) return e;
     L.ready = true;
   }
@@ -249,11 +296,11 @@ cudaError_t lanes_for_current_device(Lanes** out) {
 }
 
 // The host-buffer forward.  serial: every copy and the kernel in order on
-// the caller's stream.  Otherwise the batch is cut into up to four chunks of
-// whole batch entries, chunk c going to lane c % 2: its inputs' host-to-device
-// copies, its forward and its output's device-to-host copy, so that one
-// chunk's copies overlap another's kernel and copies in the two directions
-// overlap each other.
+// the caller's stream.  Otherwise the batch is cut into up to kLanes chunks
+// of whole batch entries, chunk c going to lane c: its inputs'
+// host-to-device copies, its forward and its output's device-to-host copy,
+// so that one chunk's copies overlap another's kernel and copies in the two
+// directions overlap each other.
 na_status forward_host_impl(const void* q_host, const void* k_host, const void* v_host, const void* rpb_host,
                             void* out_host, void* workspace, size_t workspace_bytes, int B, int heads, int H,
                             int W, int d, int ksize, na_dtype dt, void* stream, bool serial) {
@@ -276,7 +323,7 @@ na_status forward_host_impl(const void* q_host, const void* k_host, const void* 
   if (rpb_host) e = cudaMemcpyAsync(ws + L.rpb, rpb_host, L.rpb_bytes, cudaMemcpyHostToDevice, cs);
   if (e != cudaSuccess) return NA_ERR_CUDA;
   const void* rpb_dev = rpb_host ? ws + L.rpb : nullptr;
-  const int chunks = serial ? 1 : (B < 4 ? B : 4);
+  const int chunks = serial ? 1 : (B < kLanes ? B : kLanes);
   if (chunks <= 1) {
     e = cudaMemcpyAsync(ws + L.q, qh, L.tensor_bytes, cudaMemcpyHostToDevice, cs);
     if (e == cudaSuccess) e = cudaMemcpyAsync(ws + L.k, kh, L.tensor_bytes, cudaMemcpyHostToDevice, cs);
@@ -290,13 +337,13 @@ na_status forward_host_impl(const void* q_host, const void* k_host, const void* 
   Lanes* ln = nullptr;
   if (lanes_for_current_device(&ln) != cudaSuccess) return NA_ERR_CUDA;
   e = cudaEventRecord(ln->fork, cs);
-  for (int i = 0; i < 2 && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(ln->s[i], ln->fork, 0);
+  for (int i = 0; i < chunks && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(ln->s[i], ln->fork, 0);
   if (e != cudaSuccess) return NA_ERR_CUDA;
   const size_t per_b = L.tensor_bytes / (size_t)B;
   for (int c = 0; c < chunks && st == NA_OK; ++c) {
     const int b0 = (int)((long long)B * c / chunks), b1 = (int)((long long)B * (c + 1) / chunks);
     const size_t off = per_b * (size_t)b0, bytes = per_b * (size_t)(b1 - b0);
-    cudaStream_t ls = ln->s[c & 1];
+    cudaStream_t ls = ln->s[c];
     e = cudaMemcpyAsync(ws + L.q + off, qh + off, bytes, cudaMemcpyHostToDevice, ls);
     if (e == cudaSuccess) e = cudaMemcpyAsync(ws + L.k + off, kh + off, bytes, cudaMemcpyHostToDevice, ls);
     if (e == cudaSuccess) e = cudaMemcpyAsync(ws + L.v + off, vh + off, bytes, cudaMemcpyHostToDevice, ls);
@@ -309,8 +356,8 @@ na_status forward_host_impl(const void* q_host, const void* k_host, const void* 
     if (st == NA_OK && cudaMemcpyAsync(oh + off, ws + L.out + off, bytes, cudaMemcpyDeviceToHost, ls) != cudaSuccess)
       st = NA_ERR_CUDA;
   }
-  // the caller's stream waits for both lanes, also after a failed enqueue
-  for (int i = 0; i < 2; ++i)
+  // the caller's stream waits for every lane used, also after a failed enqueue
+  for (int i = 0; i < chunks; ++i)
     if (cudaEventRecord(ln->join[i], ln->s[i]) != cudaSuccess || cudaStreamWaitEvent(cs, ln->join[i], 0) != cudaSuccess)
       st = NA_ERR_CUDA;
   return st;

@@ -35,6 +35,13 @@ na_status forward_host_serial(const void* q_host, const void* k_host, const void
                               void* out_host, void* workspace, size_t workspace_bytes, int B, int heads, int H,
                               int W, int d, int ksize, na_dtype dt, void* stream);
 
+// SASA (na2d_sasa.cu): the zero-padded copies of q, k, v and the padded
+// output live in the caller's workspace (four 256-byte aligned parts).
+size_t sasa_workspace_bytes(const Shape& s, size_t es);
+cudaError_t launch_sasa_pad(const void* q, const void* k, const void* v, void* workspace, const Shape& s, size_t es,
+                            cudaStream_t st, void** qp, void** kp, void** vp, void** outp);
+cudaError_t launch_sasa_crop(const void* outp, void* out, const Shape& s, size_t es, cudaStream_t st);
+
 // Tensor-core fused forward (na2d_tc.cu), fp16/bf16.
 bool forward_tc_supported(const Shape& s, na_dtype dt);
 cudaError_t launch_forward_tc(const void* q, const void* k, const void* v, const void* rpb,

@@ -25,7 +25,7 @@ EXPORTS = (
     "na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward",
     "na2d_forward_host_workspace_bytes", "na2d_forward_host", "na2d_forward_host_noalloc", "na2d_forward_kernel",
     "na2d_device_status", "na2d_debug_timeout_probe", "na_status_str",
-    "na2d_backward_workspace_bytes", "na2d_backward",
+    "na2d_backward_workspace_bytes", "na2d_backward", "na2d_sasa_workspace_bytes", "na2d_sasa_forward",
 )
 
 
@@ -63,13 +63,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.na2d_backward_workspace_bytes.argtypes = [*shape, i]
         lib.na2d_backward_workspace_bytes.restype = sz
         lib.na2d_backward.argtypes = [vp] * 10 + [sz, *shape, i, vp]
+        lib.na2d_sasa_workspace_bytes.argtypes = [*shape, i]
+        lib.na2d_sasa_workspace_bytes.restype = sz
+        lib.na2d_sasa_forward.argtypes = [vp] * 6 + [sz, *shape, i, vp]
         lib.na2d_device_status.argtypes = [vp]
         lib.na2d_debug_timeout_probe.argtypes = [ctypes.c_uint, vp]
         lib.na_status_str.argtypes = [i]
         lib.na_status_str.restype = ctypes.c_char_p
         for name in ("na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward",
                      "na2d_forward_host", "na2d_forward_host_noalloc", "na2d_forward_kernel", "na2d_device_status",
-                     "na2d_debug_timeout_probe", "na2d_backward"):
+                     "na2d_debug_timeout_probe", "na2d_backward", "na2d_sasa_forward"):
             getattr(lib, name).restype = i
         _lib = lib
         return lib
@@ -181,6 +184,27 @@ def backward(q, k, v, rpb, dout, ksize: int, with_rpb_grad: bool = True, workspa
                              _ptr(drpb), _ptr(workspace), workspace.numel() * workspace.element_size(),
                              B, heads, H, W, d, ksize, _DT[q.dtype], _stream(q)), "na2d_backward")
     return dq, dk, dv, drpb
+
+
+def sasa_forward(q, k, v, rpb, ksize: int, out=None, workspace=None):
+    """SASA, the centred window over a zero-padded map (na2d_sasa_forward):
+    returns out [B, heads, H, W, d]."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype)
+    if rpb is not None:
+        _need(rpb, "rpb", q.dtype)
+    B, heads, H, W, d = _dims(q)
+    out = torch.empty_like(q) if out is None else out
+    _need(out, "out", q.dtype)
+    lib = load_library()
+    need = int(lib.na2d_sasa_workspace_bytes(B, heads, H, W, d, ksize, _DT[q.dtype]))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace")
+    _check(lib.na2d_sasa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(rpb), _ptr(out), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), B, heads, H, W, d, ksize,
+                                 _DT[q.dtype], _stream(q)), "na2d_sasa_forward")
+    return out
 
 
 def host_workspace_bytes(B, heads, H, W, d, ksize, dtype) -> int:
