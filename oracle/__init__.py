@@ -13,6 +13,7 @@ from .na2d_oracle import (  # noqa: F401
     av,
     backward,
     sasa_forward,
+    block_forward,
     window_start,
     max_threads,
 )

@@ -232,3 +232,42 @@ def sasa_forward(q, k, v, rpb, ks: int, nthreads: int = 0) -> np.ndarray:
     _load().na2d_oracle_sasa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(rpb), _ptr(out), B, heads, H, W, d, ks,
                                      nthreads)
     return out
+
+
+def _round_to(a, dtype_name):
+    """a rounded to fp16 / bf16 (round-to-nearest-even), back in float64."""
+    if dtype_name in (None, "f32"):
+        return a
+    import torch
+
+    t = {"f16": torch.float16, "bf16": torch.bfloat16}[dtype_name]
+    return torch.from_numpy(np.ascontiguousarray(a)).to(t).double().numpy()
+
+
+def block_forward(x, wqkv, bqkv, wo, bo, rpb, heads: int, ks: int, store=None, nthreads: int = 0):
+    """An NA block (NAT App. A.1: linear projections for queries, keys and
+    values, NA, a final linear projection; Qiita "計算量": 4hwd^2 + 2hwdk^2):
+
+        qkv = x Wqkv + bqkv          x [B, H, W, C], Wqkv [C, 3C]
+        q, k, v = the three C-channel thirds of qkv, each as heads x dh
+        o = NA_ks(q, k, v, rpb)      per head
+        y = o Wo + bo                o as [B, H, W, heads * dh], Wo [C, C]
+
+    store: None for plain float64, or "f16" / "bf16": q, k, v and o are
+    rounded to that type where a 16-bit model stores them, and y at the end.
+    Returns y [B, H, W, C]."""
+    x, wqkv, wo = (np.asarray(_f64(t)) for t in (x, wqkv, wo))
+    bqkv = None if bqkv is None else np.asarray(_f64(bqkv))
+    bo = None if bo is None else np.asarray(_f64(bo))
+    B, H, W, C = x.shape
+    dh = C // heads
+    qkv = x.reshape(-1, C) @ wqkv
+    if bqkv is not None:
+        qkv = qkv + bqkv
+    qkv = _round_to(qkv, store).reshape(B, H, W, 3, heads, dh)
+    q, k, v = (np.ascontiguousarray(qkv[:, :, :, s].transpose(0, 3, 1, 2, 4)) for s in range(3))
+    o = _round_to(forward(q, k, v, rpb, ks, nthreads), store)  # [B, heads, H, W, dh]
+    y = o.transpose(0, 2, 3, 1, 4).reshape(-1, C) @ wo
+    if bo is not None:
+        y = y + bo
+    return _round_to(y, store).reshape(B, H, W, C)

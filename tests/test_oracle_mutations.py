@@ -11,6 +11,7 @@ import oracle
 from oracle import na2d_oracle as ora
 from tests import test_oracle_backward_pins as bwd_pins
 from tests import test_oracle_pins as pins
+from tests import test_oracle_block_pins as block_pins
 from tests import test_oracle_sasa_pins as sasa_pins
 
 MUTATIONS = {
@@ -126,4 +127,36 @@ def test_planted_sasa_mistake_is_caught(mutation, tmp_path):
                 fn(**kwargs)
             except Exception:  # an assertion, or an error a pin provokes
                 failed.append(name)
+    assert failed, f"no pin caught the planted mistake: {mutation}"
+
+
+# Slips in the NA block (a Python function of the oracle), each checked
+# against the block pins.
+BLOCK_MUTATIONS = {
+    "q and k swapped in the split": ("q, k, v = (np.ascontiguousarray(qkv[:, :, :, s]",
+                                     "k, q, v = (np.ascontiguousarray(qkv[:, :, :, s]"),
+    "heads and channels swapped in the split": ("qkv = _round_to(qkv, store).reshape(B, H, W, 3, heads, dh)",
+                                                "qkv = _round_to(qkv, store).reshape(B, H, W, 3, dh, heads).swapaxes(4, 5)"),
+    "output bias dropped": ("        y = y + bo\n", "        y = y\n"),
+    "heads concatenated in the wrong order": ("y = o.transpose(0, 2, 3, 1, 4).reshape(-1, C) @ wo",
+                                              "y = o[:, ::-1].transpose(0, 2, 3, 1, 4).reshape(-1, C) @ wo"),
+}
+
+
+@pytest.mark.parametrize("mutation", sorted(BLOCK_MUTATIONS))
+def test_planted_block_mistake_is_caught(mutation, monkeypatch):
+    import textwrap
+
+    old, new = BLOCK_MUTATIONS[mutation]
+    src = textwrap.dedent(inspect.getsource(ora.block_forward))
+    assert src.count(old) == 1, f"mutation anchor not found once: {mutation}"
+    scope = dict(vars(ora))
+    exec(compile(src.replace(old, new), "<mutant>", "exec"), scope)
+    monkeypatch.setattr(oracle, "block_forward", scope["block_forward"])
+    failed = []
+    for name, fn, kwargs in _pin_cases(block_pins):
+        try:
+            fn(**kwargs)
+        except Exception:  # an assertion, or an error a pin provokes
+            failed.append(name)
     assert failed, f"no pin caught the planted mistake: {mutation}"
