@@ -24,7 +24,8 @@
  *
  * Ownership: the caller allocates and owns every buffer.  Device pointers
  * must point to device memory of the current CUDA device and be 16-byte
- * aligned.  The library allocates no memory in any call; it keeps only a
+ * aligned.  The library allocates no memory in any call (cuBLAS allocates
+ * its handle's state at the first na2d_block_forward on a device); it keeps only a
  * per-device status word (a static device variable), encoded TMA
  * descriptors passed by value to its kernels, and the fixed staging array
  * of na2d_forward_host_noalloc (a static device variable).
@@ -154,13 +155,40 @@ na_status na2d_sasa_forward(const void *q, const void *k, const void *v, const v
                             na_dtype dt, void *stream);
 
 /*
+ * An NA block: the query/key/value projection, neighborhood attention, and
+ * the output projection (NAT App. A.1: linear projections for queries,
+ * keys and values followed by a final linear projection; the Qiita
+ * write-up's "計算量" counts the block as 4hwd^2 + 2hwdk^2):
+ *
+ *   qkv = x Wqkv + bqkv,  q | k | v = its three C-channel thirds (each heads x dh),
+ *   o = NA_ks(q, k, v, rpb) per head,  y = o Wo + bo,   C = heads * dh.
+ *
+ * x, y: [B][H][W][C]; wqkv: [C][3C]; bqkv: [3C] or NULL; wo: [C][C]; bo: [C]
+ * or NULL; rpb as na2d_forward; all of type dt (dh and ksize as na2d_forward's
+ * d and ksize).  The projections run in cuBLAS with float32 accumulation;
+ * q, k, v and o are stored in dt between the steps, y is rounded to dt.
+ * workspace: a 256-byte aligned device buffer of at least
+ * na2d_block_workspace_bytes() bytes that the caller owns (it also serves
+ * as cuBLAS's workspace); its contents on entry do not matter.  The first
+ * call on a device creates a cuBLAS handle for it (cuBLAS allocates its
+ * own small state then) and keeps it; make that call before any stream
+ * capture.
+ */
+size_t na2d_block_workspace_bytes(int B, int H, int W, int heads, int dh, int ksize, na_dtype dt);
+na_status na2d_block_forward(const void *x, const void *wqkv, const void *bqkv, const void *wo, const void *bo,
+                             const void *rpb, void *y, void *workspace, size_t workspace_bytes,
+                             int B, int H, int W, int heads, int dh, int ksize,
+                             na_dtype dt, void *stream);
+
+/*
  * na2d_forward from HOST buffers: copies q, k, v (and rpb when not NULL)
  * host-to-device into the caller's device workspace, runs na2d_forward and
  * copies the result back to out_host, one cudaMemcpyAsync per buffer and
  * batch chunk.  With B >= 2 the batch is cut into up to four chunks of whole
  * batch entries, each on a stream of the library's own, forked from and
- * joined back to `stream` with events, so that one chunk's copies overlap
- * another chunk's kernel; the call is still ordered on `stream` as one
+ * joined back to `stream` with events; the chunks' input copies run one
+ * after another, so that one chunk's kernel and output copy overlap the next
+ * chunk's input copies.  The call is still ordered on `stream` as one
  * operation.  The library creates those four streams and their events on
  * the first such call on a device and keeps them; make that first call
  * before any stream capture.  Pinned host memory makes the copies

@@ -160,3 +160,15 @@ def test_sasa_arguments(lib):
     assert lib.na2d_sasa_forward(None, FAKE, FAKE, None, FAKE, FAKE, need, 1, 1, 5, 6, 32, 7, na2d.NA_BF16,
                                  None) == na2d.NA_ERR_INVALID_ARG
     assert lib.na2d_sasa_forward(*args, None, 0, 0, 1, 5, 6, 32, 7, na2d.NA_BF16, None) == na2d.NA_OK
+
+
+def test_block_arguments(lib):
+    need = lib.na2d_block_workspace_bytes(2, 8, 8, 2, 32, 3, na2d.NA_BF16)
+    assert need > 2 * 8 * 8 * 64 * (3 * 4 + 5 * 2 + 4)
+    assert lib.na2d_block_workspace_bytes(2, 8, 8, 2, 48, 3, na2d.NA_BF16) == 0
+    a = (FAKE, FAKE, None, FAKE, None, None, FAKE)
+    assert lib.na2d_block_forward(*a, FAKE, need - 1, 2, 8, 8, 2, 32, 3, na2d.NA_BF16, None) == na2d.NA_ERR_INVALID_ARG
+    assert lib.na2d_block_forward(*a, FAKE + 16, need, 2, 8, 8, 2, 32, 3, na2d.NA_BF16, None) == na2d.NA_ERR_INVALID_ARG
+    assert lib.na2d_block_forward(None, FAKE, None, FAKE, None, None, FAKE, FAKE, need, 2, 8, 8, 2, 32, 3,
+                                  na2d.NA_BF16, None) == na2d.NA_ERR_INVALID_ARG
+    assert lib.na2d_block_forward(*a, None, 0, 0, 8, 8, 2, 32, 3, na2d.NA_BF16, None) == na2d.NA_OK

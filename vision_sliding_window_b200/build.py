@@ -5,7 +5,8 @@
 Each .cu file under csrc/ is compiled with
 `-gencode arch=compute_100a,code=sm_100a -O3 -lineinfo`, then linked into a
 shared object with the CUDA runtime linked statically (so loading the
-library needs no CUDA driver; only calling it does).  Only the symbols of
+library needs no CUDA driver; only calling it does) and cuBLAS linked
+dynamically (for the NA block's two projections).  Only the symbols of
 include/na2d.h are exported.
 """
 from __future__ import annotations
@@ -78,7 +79,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         objs = list(ex.map(compile_one, _sources()))
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [cc, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
+    cmd = [cc, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs, "-lcublas"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

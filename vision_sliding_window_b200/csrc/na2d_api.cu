@@ -229,6 +229,32 @@ NA_EXPORT na_status na2d_sasa_forward(const void* q, const void* k, const void* 
   return from_cuda(launch_sasa_crop(outp, out, s, es, cs));
 }
 
+NA_EXPORT size_t na2d_block_workspace_bytes(int B, int H, int W, int heads, int dh, int ksize, na_dtype dt) {
+  Shape s;
+  if (check_dtype(dt) != NA_OK || check_shape(B, heads, H, W, dh, ksize, true, &s) != NA_OK) return 0;
+  if ((long long)B * H * W >= (1ll << 31) || (long long)heads * dh * 3 >= (1ll << 31)) return 0;
+  return block_workspace_bytes(B, H, W, heads, dh, elem_size(dt));
+}
+
+NA_EXPORT na_status na2d_block_forward(const void* x, const void* wqkv, const void* bqkv, const void* wo,
+                                       const void* bo, const void* rpb, void* y, void* workspace,
+                                       size_t workspace_bytes, int B, int H, int W, int heads, int dh, int ksize,
+                                       na_dtype dt, void* stream) {
+  Shape s;
+  na_status st = check_dtype(dt);
+  if (st == NA_OK) st = check_shape(B, heads, H, W, dh, ksize, true, &s);
+  if (st != NA_OK) return st;
+  if (s.queries() == 0) return NA_OK;
+  if ((long long)B * H * W >= (1ll << 31) || (long long)heads * dh * 3 >= (1ll << 31)) return NA_ERR_INVALID_ARG;
+  for (const void* ptr : {x, wqkv, wo, (const void*)y})
+    if (!ptr || !aligned16(ptr)) return NA_ERR_INVALID_ARG;
+  for (const void* ptr : {bqkv, bo, rpb})
+    if (ptr && !aligned16(ptr)) return NA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NA_ERR_INVALID_ARG;
+  if (workspace_bytes < block_workspace_bytes(B, H, W, heads, dh, elem_size(dt))) return NA_ERR_INVALID_ARG;
+  return run_block(x, wqkv, bqkv, wo, bo, rpb, y, workspace, B, H, W, heads, dh, ksize, dt, (cudaStream_t)stream);
+}
+
 namespace {
 struct HostLayout {
   size_t q, k, v, rpb, out, total, tensor_bytes, rpb_bytes;
@@ -270,7 +296,7 @@ namespace {
 constexpr int kLanes = 4;
 struct Lanes {
   cudaStream_t s[kLanes];
-  cudaEvent_t fork, join[kLanes];
+  cudaEvent_t fork, join[kLanes], in_done[kLanes];
   bool ready;
 };
 constexpr int kMaxDevices = 64;
@@ -286,8 +312,10 @@ cudaError_t lanes_for_current_device(Lanes** out) {
   if (!L.ready) {
     for (int i = 0; i < kLanes && e == cudaSuccess; ++i) e = cudaStreamCreateWithFlags(&L.s[i], cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L.fork, cudaEventDisableTiming);
-    for (int i = 0; i < kLanes && e == cudaSuccess; ++i)
+    for (int i = 0; i < kLanes && e == cudaSuccess; ++i) {
       e = cudaEventCreateWithFlags(&L.join[i], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L.in_done[i], cudaEventDisableTiming);
+    }
     if (e != cudaSuccess) return e;
     L.ready = true;
   }
@@ -344,9 +372,15 @@ na_status forward_host_impl(const void* q_host, const void* k_host, const void* 
     const int b0 = (int)((long long)B * c / chunks), b1 = (int)((long long)B * (c + 1) / chunks);
     const size_t off = per_b * (size_t)b0, bytes = per_b * (size_t)(b1 - b0);
     cudaStream_t ls = ln->s[c];
-    e = cudaMemcpyAsync(ws + L.q + off, qh + off, bytes, cudaMemcpyHostToDevice, ls);
+    // the chunks' input copies run one after another, each at the link's
+    // full rate, so that chunk c's kernel starts as soon as its own inputs
+    // are in (copies running side by side would share the link and land
+    // together)
+    e = c > 0 ? cudaStreamWaitEvent(ls, ln->in_done[c - 1], 0) : cudaSuccess;
+    if (e == cudaSuccess) e = cudaMemcpyAsync(ws + L.q + off, qh + off, bytes, cudaMemcpyHostToDevice, ls);
     if (e == cudaSuccess) e = cudaMemcpyAsync(ws + L.k + off, kh + off, bytes, cudaMemcpyHostToDevice, ls);
     if (e == cudaSuccess) e = cudaMemcpyAsync(ws + L.v + off, vh + off, bytes, cudaMemcpyHostToDevice, ls);
+    if (e == cudaSuccess) e = cudaEventRecord(ln->in_done[c], ls);
     if (e != cudaSuccess) {
       st = NA_ERR_CUDA;
       break;

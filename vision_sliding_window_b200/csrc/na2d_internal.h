@@ -42,6 +42,12 @@ cudaError_t launch_sasa_pad(const void* q, const void* k, const void* v, void* w
                             cudaStream_t st, void** qp, void** kp, void** vp, void** outp);
 cudaError_t launch_sasa_crop(const void* outp, void* out, const Shape& s, size_t es, cudaStream_t st);
 
+// NA block (na2d_block.cu): projections in cuBLAS around na2d_forward.
+size_t block_workspace_bytes(int B, int H, int W, int heads, int dh, size_t es);
+na_status run_block(const void* x, const void* wqkv, const void* bqkv, const void* wo, const void* bo, const void* rpb,
+                    void* y, void* workspace, int B, int H, int W, int heads, int dh, int ks, na_dtype dt,
+                    cudaStream_t st);
+
 // Tensor-core fused forward (na2d_tc.cu), fp16/bf16.
 bool forward_tc_supported(const Shape& s, na_dtype dt);
 cudaError_t launch_forward_tc(const void* q, const void* k, const void* v, const void* rpb,

@@ -129,3 +129,21 @@ def sample_points(w: Workload, n: int, seed: int = 1):
         ], dim=1)
         pts = torch.cat([pts, rnd])
     return pts[:max(n, len(fixed))]
+
+
+def make_block_inputs(B: int, H: int, W: int, heads: int, dh: int, ks: int, dtype="bf16", *, seed: int = 0):
+    """Synthetic weights and input of an NA block (x [B, H, W, C], Wqkv [C, 3C],
+    bqkv [3C], Wo [C, C], bo [C], rpb [heads, 2ks-1, 2ks-1], C = heads * dh):
+    x ~ N(0, 1), weights ~ N(0, 1/C), biases ~ N(0, 0.1^2), rpb ~ N(0, 0.02^2),
+    from one CPU generator in that order, then rounded to `dtype`."""
+    tdt = DTYPES[dtype] if isinstance(dtype, str) else dtype
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    C = heads * dh
+    x = torch.randn((B, H, W, C), generator=g)
+    wqkv = torch.randn((C, 3 * C), generator=g) / C ** 0.5
+    bqkv = torch.randn(3 * C, generator=g) * 0.1
+    wo = torch.randn((C, C), generator=g) / C ** 0.5
+    bo = torch.randn(C, generator=g) * 0.1
+    rpb = torch.randn((heads, 2 * ks - 1, 2 * ks - 1), generator=g) * 0.02
+    return tuple(t.to(tdt) for t in (x, wqkv, bqkv, wo, bo, rpb))

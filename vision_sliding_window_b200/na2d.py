@@ -26,6 +26,7 @@ EXPORTS = (
     "na2d_forward_host_workspace_bytes", "na2d_forward_host", "na2d_forward_host_noalloc", "na2d_forward_kernel",
     "na2d_device_status", "na2d_debug_timeout_probe", "na_status_str",
     "na2d_backward_workspace_bytes", "na2d_backward", "na2d_sasa_workspace_bytes", "na2d_sasa_forward",
+    "na2d_block_workspace_bytes", "na2d_block_forward",
 )
 
 
@@ -66,13 +67,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.na2d_sasa_workspace_bytes.argtypes = [*shape, i]
         lib.na2d_sasa_workspace_bytes.restype = sz
         lib.na2d_sasa_forward.argtypes = [vp] * 6 + [sz, *shape, i, vp]
+        lib.na2d_block_workspace_bytes.argtypes = [*shape, i]
+        lib.na2d_block_workspace_bytes.restype = sz
+        lib.na2d_block_forward.argtypes = [vp] * 8 + [sz, *shape, i, vp]
         lib.na2d_device_status.argtypes = [vp]
         lib.na2d_debug_timeout_probe.argtypes = [ctypes.c_uint, vp]
         lib.na_status_str.argtypes = [i]
         lib.na_status_str.restype = ctypes.c_char_p
         for name in ("na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward",
                      "na2d_forward_host", "na2d_forward_host_noalloc", "na2d_forward_kernel", "na2d_device_status",
-                     "na2d_debug_timeout_probe", "na2d_backward", "na2d_sasa_forward"):
+                     "na2d_debug_timeout_probe", "na2d_backward", "na2d_sasa_forward", "na2d_block_forward"):
             getattr(lib, name).restype = i
         _lib = lib
         return lib
@@ -205,6 +209,35 @@ def sasa_forward(q, k, v, rpb, ksize: int, out=None, workspace=None):
                                  workspace.numel() * workspace.element_size(), B, heads, H, W, d, ksize,
                                  _DT[q.dtype], _stream(q)), "na2d_sasa_forward")
     return out
+
+
+def block_forward(x, wqkv, bqkv, wo, bo, rpb, heads: int, ksize: int, y=None, workspace=None):
+    """An NA block (na2d_block_forward): y = NA(x Wqkv + bqkv) Wo + bo, x and y
+    [B, H, W, heads * dh]."""
+    for t, n in ((x, "x"), (wqkv, "wqkv"), (wo, "wo")):
+        _need(t, n, x.dtype)
+    for t, n in ((bqkv, "bqkv"), (bo, "bo"), (rpb, "rpb")):
+        if t is not None:
+            _need(t, n, x.dtype)
+    if x.dim() != 4:
+        raise ValueError("x must be [B, H, W, C]")
+    B, H, W, C = (int(s) for s in x.shape)
+    if C % heads:
+        raise ValueError("C must be a multiple of heads")
+    dh = C // heads
+    y = torch.empty_like(x) if y is None else y
+    _need(y, "y", x.dtype)
+    lib = load_library()
+    need = int(lib.na2d_block_workspace_bytes(B, H, W, heads, dh, ksize, _DT[x.dtype]))
+    if need == 0:
+        raise NA2DError(NA_ERR_INVALID_ARG, "na2d_block_forward")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    _need(workspace, "workspace")
+    _check(lib.na2d_block_forward(_ptr(x), _ptr(wqkv), _ptr(bqkv), _ptr(wo), _ptr(bo), _ptr(rpb), _ptr(y),
+                                  _ptr(workspace), workspace.numel() * workspace.element_size(), B, H, W, heads, dh,
+                                  ksize, _DT[x.dtype], _stream(x)), "na2d_block_forward")
+    return y
 
 
 def host_workspace_bytes(B, heads, H, W, d, ksize, dtype) -> int:
