@@ -14,6 +14,7 @@ from .na2d_oracle import (  # noqa: F401
     backward,
     sasa_forward,
     block_forward,
+    nd_forward,
     window_start,
     max_threads,
 )

@@ -360,6 +360,85 @@ void na2d_oracle_sasa_forward(const double *q, const double *k, const double *v,
     }
 }
 
+/*
+ * Neighborhood attention over 1, 2 or 3 axes with dilation.  The NATTEN
+ * library supports "1D to 3D" NA (Qiita write-up, section "NATTEN"; NAT
+ * Sec. 3.2: 1D and 2D data), and the DiNAT abstract names a dilated NA; the
+ * pages give no formula for dilation.  Reading: a dilation dl on an axis of
+ * length L splits it into dl interleaved sub-grids (positions = r mod dl),
+ * and a query attends within its own sub-grid with NA's clamped window of
+ * ka positions:
+ *
+ *   r = i mod dl,  i' = i div dl,  L' = ceil((L - r) / dl),
+ *   start' = clamp(i' - ka/2, 0, L' - ka),  keys at r + (start' + t) dl,
+ *   bias index (start' + t) - i' + ka - 1 on that axis.
+ *
+ * 1D and 2D are the cases with unit extents and kernel sizes on the leading
+ * axes; with dl = 1 every axis is plain NA.  Layouts:
+ * q, k, v, out [B][heads][L0][L1][L2][d]; rpb [heads][2k0-1][2k1-1][2k2-1]
+ * or NULL.  Every sub-grid must hold a window: floor(La / dla) >= ka.
+ */
+static long axis_start(long i, long L, long ka, long dl, long *r, long *ip)
+{
+    long rr = i % dl, ii = i / dl, Lp = (L - rr + dl - 1) / dl;
+    long s = ii - ka / 2;
+    if (s < 0) s = 0;
+    if (s > Lp - ka) s = Lp - ka;
+    *r = rr;
+    *ip = ii;
+    return s;
+}
+
+void na2d_oracle_nd_forward(const double *q, const double *k, const double *v, const double *rpb, double *out,
+                            long B, long heads, long L0, long L1, long L2, long d,
+                            long k0, long k1, long k2, long dl0, long dl1, long dl2, int nthreads)
+{
+    long rows = B * heads * L0 * L1, nn = k0 * k1 * k2;
+    long s0 = 2 * k0 - 1, s1 = 2 * k1 - 1, s2 = 2 * k2 - 1;
+    double scale = 1.0 / sqrt((double)d);
+#pragma omp parallel num_threads(threads_for(nthreads))
+    {
+        double *A = (double *)malloc(sizeof(double) * (size_t)nn);
+        long *pos = (long *)malloc(sizeof(long) * (size_t)nn);
+#pragma omp for schedule(dynamic)
+        for (long row = 0; row < rows; row++) {
+            long i1 = row % L1, t0 = row / L1, i0 = t0 % L0, bh = t0 / L0, h = bh % heads;
+            for (long i2 = 0; i2 < L2; i2++) {
+                long r0, r1, r2, p0, p1, p2;
+                long st0 = axis_start(i0, L0, k0, dl0, &r0, &p0);
+                long st1 = axis_start(i1, L1, k1, dl1, &r1, &p1);
+                long st2 = axis_start(i2, L2, k2, dl2, &r2, &p2);
+                size_t map = (size_t)bh * L0 * L1 * L2;
+                const double *qv = q + (map + ((size_t)i0 * L1 + i1) * L2 + i2) * d;
+                long n = 0;
+                for (long a = 0; a < k0; a++)
+                    for (long b = 0; b < k1; b++)
+                        for (long c = 0; c < k2; c++, n++) {
+                            long j0 = r0 + (st0 + a) * dl0, j1 = r1 + (st1 + b) * dl1, j2 = r2 + (st2 + c) * dl2;
+                            long kp = (long)(map + ((size_t)j0 * L1 + j1) * L2 + j2);
+                            const double *kv = k + (size_t)kp * d;
+                            double dot = 0.0;
+                            for (long x = 0; x < d; x++) dot += qv[x] * kv[x];
+                            if (rpb)
+                                dot += rpb[(((size_t)h * s0 + (st0 + a - p0 + k0 - 1)) * s1 +
+                                            (st1 + b - p1 + k1 - 1)) * s2 + (st2 + c - p2 + k2 - 1)];
+                            A[n] = dot;
+                            pos[n] = kp;
+                        }
+                softmax_row(A, nn, scale);
+                double *o = out + (map + ((size_t)i0 * L1 + i1) * L2 + i2) * d;
+                for (long x = 0; x < d; x++) o[x] = 0.0;
+                for (long m = 0; m < nn; m++) {
+                    const double *vv = v + (size_t)pos[m] * d;
+                    for (long x = 0; x < d; x++) o[x] += A[m] * vv[x];
+                }
+            }
+        }
+        free(A);
+        free(pos);
+    }
+}
+
 int na2d_oracle_max_threads(void)
 {
     return threads_for(0);

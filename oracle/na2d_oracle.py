@@ -56,6 +56,7 @@ def _load():
             )
             lib.na2d_oracle_backward.argtypes = [_D] * 9 + [_L] * 6 + [ctypes.c_int]
             lib.na2d_oracle_sasa_forward.argtypes = [_D] * 5 + [_L] * 6 + [ctypes.c_int]
+            lib.na2d_oracle_nd_forward.argtypes = [_D] * 5 + [_L] * 12 + [ctypes.c_int]
             lib.na2d_oracle_max_threads.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -76,6 +77,7 @@ class swapped_library:
         for fn in ("na2d_oracle_window_start", "na2d_oracle_qk_rpb", "na2d_oracle_softmax",
                    "na2d_oracle_av", "na2d_oracle_forward", "na2d_oracle_forward_rows",
                    "na2d_oracle_forward_points", "na2d_oracle_backward", "na2d_oracle_sasa_forward",
+                   "na2d_oracle_nd_forward",
                    "na2d_oracle_max_threads"):
             src, dst = getattr(self._saved, fn), getattr(lib, fn)
             dst.argtypes, dst.restype = src.argtypes, src.restype
@@ -271,3 +273,29 @@ def block_forward(x, wqkv, bqkv, wo, bo, rpb, heads: int, ks: int, store=None, n
     if bo is not None:
         y = y + bo
     return _round_to(y, store).reshape(B, H, W, C)
+
+
+def nd_forward(q, k, v, rpb, ks, dilation=None, nthreads: int = 0) -> np.ndarray:
+    """NA over the trailing 1, 2 or 3 spatial axes of q [B, heads, *spatial, d]
+    with per-axis kernel sizes ks and dilations (the sub-grid reading: a
+    query attends within the positions congruent to it mod the dilation, with
+    NA's clamped window there).  rpb [heads, *(2k - 1)] or None."""
+    q, k, v, rpb = _f64(q), _f64(k), _f64(v), _f64(rpb)
+    nsp = q.ndim - 3
+    if nsp not in (1, 2, 3):
+        raise ValueError("q must be [B, heads, *spatial, d] with 1-3 spatial axes")
+    ks = tuple(ks) if hasattr(ks, "__len__") else (ks,) * nsp
+    dilation = tuple(dilation) if dilation is not None else (1,) * nsp
+    B, heads, d = q.shape[0], q.shape[1], q.shape[-1]
+    L = (1,) * (3 - nsp) + tuple(q.shape[2:-1])
+    kk = (1,) * (3 - nsp) + ks
+    dl = (1,) * (3 - nsp) + dilation
+    for La, ka, da in zip(L, kk, dl):
+        if ka % 2 != 1 or da < 1 or La // da < ka:
+            raise ValueError(f"axis of length {La}: kernel {ka} (odd) and dilation {da} need L // dilation >= kernel")
+    if rpb is not None:
+        rpb = np.ascontiguousarray(rpb.reshape(heads, 2 * kk[0] - 1, 2 * kk[1] - 1, 2 * kk[2] - 1))
+    out = np.empty_like(q)
+    _load().na2d_oracle_nd_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(rpb), _ptr(out), B, heads, *L, d, *kk, *dl,
+                                   nthreads)
+    return out

@@ -12,6 +12,7 @@ from oracle import na2d_oracle as ora
 from tests import test_oracle_backward_pins as bwd_pins
 from tests import test_oracle_pins as pins
 from tests import test_oracle_block_pins as block_pins
+from tests import test_oracle_nd_pins as nd_pins
 from tests import test_oracle_sasa_pins as sasa_pins
 
 MUTATIONS = {
@@ -159,4 +160,35 @@ def test_planted_block_mistake_is_caught(mutation, monkeypatch):
             fn(**kwargs)
         except Exception:  # an assertion, or an error a pin provokes
             failed.append(name)
+    assert failed, f"no pin caught the planted mistake: {mutation}"
+
+
+# Slips in NA over 1-3 axes with dilation, each checked against its pins.
+ND_MUTATIONS = {
+    "dilation ignored in the key positions": (
+        "long j0 = r0 + (st0 + a) * dl0, j1 = r1 + (st1 + b) * dl1, j2 = r2 + (st2 + c) * dl2;",
+        "long j0 = r0 + (st0 + a), j1 = r1 + (st1 + b), j2 = r2 + (st2 + c);"),
+    "sub-grid length rounded down": ("long rr = i % dl, ii = i / dl, Lp = (L - rr + dl - 1) / dl;",
+                                     "long rr = i % dl, ii = i / dl, Lp = L / dl;"),
+    "bias as if every window were centred": ("(st1 + b - p1 + k1 - 1)) * s2",
+                                             "(b + k1 / 2)) * s2"),
+    "window not clamped": ("    if (s > Lp - ka) s = Lp - ka;\n    *r = rr;", "    *r = rr;"),
+    "axes 1 and 2 swapped in the bias": ("(st1 + b - p1 + k1 - 1)) * s2 + (st2 + c - p2 + k2 - 1)]",
+                                         "(st2 + c - p2 + k2 - 1)) * s2 + (st1 + b - p1 + k1 - 1)]"),
+}
+
+
+@pytest.mark.parametrize("mutation", sorted(ND_MUTATIONS))
+def test_planted_nd_mistake_is_caught(mutation, tmp_path):
+    old, new = ND_MUTATIONS[mutation]
+    text = ora.source_text()
+    assert text.count(old) == 1, f"mutation anchor not found once: {mutation}"
+    lib = ora.compile_variant(text.replace(old, new), str(tmp_path / "mutant.so"))
+    failed = []
+    with ora.swapped_library(lib):
+        for name, fn, kwargs in _pin_cases(nd_pins):
+            try:
+                fn(**kwargs)
+            except Exception:  # an assertion, or an error a pin provokes
+                failed.append(name)
     assert failed, f"no pin caught the planted mistake: {mutation}"
