@@ -181,6 +181,31 @@ na_status na2d_block_forward(const void *x, const void *wqkv, const void *bqkv, 
                              na_dtype dt, void *stream);
 
 /*
+ * Neighborhood attention over 1, 2 or 3 axes with dilation: NATTEN's NA
+ * "from 1D to 3D" (Qiita write-up, section "NATTEN"; NAT Sec. 3.2) and the
+ * dilated NA of DiNAT.  The pages give no formula for dilation; this call
+ * reads a dilation dl as splitting an axis into dl interleaved sub-grids
+ * (positions congruent mod dl), a query attending within its own sub-grid
+ * with NA's clamped window of k positions:
+ *
+ *   r = i mod dl, i' = i div dl, L' = ceil((L - r) / dl),
+ *   start' = clamp(i' - k/2, 0, L' - k), keys at r + (start' + t) dl,
+ *   bias index (start' + t) - i' + k - 1 on that axis.
+ *
+ * q, k, v, out: [B][heads][L0][L1][L2][d]; rpb: [heads][2k0-1][2k1-1][2k2-1]
+ * or NULL; all of type dt.  1D and 2D NA are the cases L0 = k0 = 1 (and
+ * L1 = k1 = 1); with every dilation 1 and L0 = k0 = 1 this is na2d_forward.
+ * Arguments: every k odd, 1 .. 63; every dilation >= 1; L / dilation >= k on
+ * every axis (each sub-grid holds a window); d in {16, 32, 64, 128}.
+ * CUDA-core kernel with the exact row maximum; float64 accumulation for
+ * NA_F32, float32 otherwise.
+ */
+na_status na_forward_nd(const void *q, const void *k, const void *v, const void *rpb, void *out,
+                        int B, int heads, int L0, int L1, int L2, int d,
+                        int k0, int k1, int k2, int dil0, int dil1, int dil2,
+                        na_dtype dt, void *stream);
+
+/*
  * na2d_forward from HOST buffers: copies q, k, v (and rpb when not NULL)
  * host-to-device into the caller's device workspace, runs na2d_forward and
  * copies the result back to out_host, one cudaMemcpyAsync per buffer and

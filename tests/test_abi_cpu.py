@@ -172,3 +172,12 @@ def test_block_arguments(lib):
     assert lib.na2d_block_forward(None, FAKE, None, FAKE, None, None, FAKE, FAKE, need, 2, 8, 8, 2, 32, 3,
                                   na2d.NA_BF16, None) == na2d.NA_ERR_INVALID_ARG
     assert lib.na2d_block_forward(*a, None, 0, 0, 8, 8, 2, 32, 3, na2d.NA_BF16, None) == na2d.NA_OK
+
+
+@pytest.mark.parametrize("kw", [dict(k2=4), dict(dil1=0), dict(L2=10, dil2=4, k2=3), dict(d=24), dict(q=None),
+                                dict(out=FAKE + 8), dict(L0=0)])
+def test_nd_rejects_bad_arguments(lib, kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, rpb=None, out=FAKE, B=1, heads=1, L0=1, L1=9, L2=12, d=32, k0=1, k1=3, k2=5,
+             dil0=1, dil1=2, dil2=2)
+    a.update(kw)
+    assert lib.na_forward_nd(*a.values(), na2d.NA_BF16, None) == na2d.NA_ERR_INVALID_ARG

@@ -255,6 +255,28 @@ NA_EXPORT na_status na2d_block_forward(const void* x, const void* wqkv, const vo
   return run_block(x, wqkv, bqkv, wo, bo, rpb, y, workspace, B, H, W, heads, dh, ksize, dt, (cudaStream_t)stream);
 }
 
+NA_EXPORT na_status na_forward_nd(const void* q, const void* k, const void* v, const void* rpb, void* out, int B,
+                                  int heads, int L0, int L1, int L2, int d, int k0, int k1, int k2, int dil0,
+                                  int dil1, int dil2, na_dtype dt, void* stream) {
+  na_status st = check_dtype(dt);
+  if (st != NA_OK) return st;
+  const int L[3] = {L0, L1, L2}, ks[3] = {k0, k1, k2}, dil[3] = {dil0, dil1, dil2};
+  if (B < 0 || heads < 0 || (d != 16 && d != 32 && d != 64 && d != 128)) return NA_ERR_INVALID_ARG;
+  long double n = (long double)B * heads;
+  for (int a = 0; a < 3; ++a) {
+    if (L[a] < 1 || ks[a] < 1 || (ks[a] & 1) == 0 || ks[a] > 63 || dil[a] < 1) return NA_ERR_INVALID_ARG;
+    if (L[a] / dil[a] < ks[a]) return NA_ERR_INVALID_ARG;  // every sub-grid holds a window
+    n *= L[a];
+  }
+  if (n * (long double)(d > ks[0] * ks[1] * ks[2] ? d : ks[0] * ks[1] * ks[2]) >= (long double)(1ll << 62))
+    return NA_ERR_INVALID_ARG;
+  if (n == 0) return NA_OK;
+  for (const void* ptr : {q, k, v, (const void*)out})
+    if (!ptr || !aligned16(ptr)) return NA_ERR_INVALID_ARG;
+  if (rpb && !aligned16(rpb)) return NA_ERR_INVALID_ARG;
+  return from_cuda(launch_forward_nd(q, k, v, rpb, out, B, heads, L, d, ks, dil, dt, (cudaStream_t)stream));
+}
+
 namespace {
 struct HostLayout {
   size_t q, k, v, rpb, out, total, tensor_bytes, rpb_bytes;

@@ -48,6 +48,11 @@ na_status run_block(const void* x, const void* wqkv, const void* bqkv, const voi
                     void* y, void* workspace, int B, int H, int W, int heads, int dh, int ks, na_dtype dt,
                     cudaStream_t st);
 
+// NA over 1-3 axes with dilation (na2d_nd.cu).
+cudaError_t launch_forward_nd(const void* q, const void* k, const void* v, const void* rpb, void* out, int B,
+                              int heads, const int (&L)[3], int d, const int (&ks)[3], const int (&dil)[3],
+                              na_dtype dt, cudaStream_t st);
+
 // Tensor-core fused forward (na2d_tc.cu), fp16/bf16.
 bool forward_tc_supported(const Shape& s, na_dtype dt);
 cudaError_t launch_forward_tc(const void* q, const void* k, const void* v, const void* rpb,

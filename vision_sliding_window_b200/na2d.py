@@ -26,7 +26,7 @@ EXPORTS = (
     "na2d_forward_host_workspace_bytes", "na2d_forward_host", "na2d_forward_host_noalloc", "na2d_forward_kernel",
     "na2d_device_status", "na2d_debug_timeout_probe", "na_status_str",
     "na2d_backward_workspace_bytes", "na2d_backward", "na2d_sasa_workspace_bytes", "na2d_sasa_forward",
-    "na2d_block_workspace_bytes", "na2d_block_forward",
+    "na2d_block_workspace_bytes", "na2d_block_forward", "na_forward_nd",
 )
 
 
@@ -70,13 +70,15 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.na2d_block_workspace_bytes.argtypes = [*shape, i]
         lib.na2d_block_workspace_bytes.restype = sz
         lib.na2d_block_forward.argtypes = [vp] * 8 + [sz, *shape, i, vp]
+        lib.na_forward_nd.argtypes = [vp] * 5 + [i] * 12 + [i, vp]
         lib.na2d_device_status.argtypes = [vp]
         lib.na2d_debug_timeout_probe.argtypes = [ctypes.c_uint, vp]
         lib.na_status_str.argtypes = [i]
         lib.na_status_str.restype = ctypes.c_char_p
         for name in ("na2d_qk_rpb", "na2d_softmax", "na2d_av", "na2d_forward",
                      "na2d_forward_host", "na2d_forward_host_noalloc", "na2d_forward_kernel", "na2d_device_status",
-                     "na2d_debug_timeout_probe", "na2d_backward", "na2d_sasa_forward", "na2d_block_forward"):
+                     "na2d_debug_timeout_probe", "na2d_backward", "na2d_sasa_forward", "na2d_block_forward",
+                     "na_forward_nd"):
             getattr(lib, name).restype = i
         _lib = lib
         return lib
@@ -238,6 +240,29 @@ def block_forward(x, wqkv, bqkv, wo, bo, rpb, heads: int, ksize: int, y=None, wo
                                   _ptr(workspace), workspace.numel() * workspace.element_size(), B, H, W, heads, dh,
                                   ksize, _DT[x.dtype], _stream(x)), "na2d_block_forward")
     return y
+
+
+def forward_nd(q, k, v, rpb, ks, dilation=None, out=None):
+    """NA over the 1-3 spatial axes of q [B, heads, *spatial, d] with per-axis
+    kernel sizes ks and dilations (na_forward_nd)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype)
+    if rpb is not None:
+        _need(rpb, "rpb", q.dtype)
+    nsp = q.dim() - 3
+    if nsp not in (1, 2, 3):
+        raise ValueError("q must be [B, heads, *spatial, d] with 1-3 spatial axes")
+    ks = tuple(ks) if hasattr(ks, "__len__") else (ks,) * nsp
+    dilation = tuple(dilation) if dilation is not None else (1,) * nsp
+    B, heads, d = int(q.shape[0]), int(q.shape[1]), int(q.shape[-1])
+    L = (1,) * (3 - nsp) + tuple(int(x) for x in q.shape[2:-1])
+    kk = (1,) * (3 - nsp) + ks
+    dl = (1,) * (3 - nsp) + dilation
+    out = torch.empty_like(q) if out is None else out
+    _need(out, "out", q.dtype)
+    _check(load_library().na_forward_nd(_ptr(q), _ptr(k), _ptr(v), _ptr(rpb), _ptr(out), B, heads, *L, d, *kk, *dl,
+                                        _DT[q.dtype], _stream(q)), "na_forward_nd")
+    return out
 
 
 def host_workspace_bytes(B, heads, H, W, d, ksize, dtype) -> int:
