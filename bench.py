@@ -60,6 +60,8 @@ def parse_args(argv=None):
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph-steps", type=int, default=250, help="steps per captured CUDA graph")
+    ap.add_argument("--api", choices=["fused", "unfused"], default="fused",
+                    help="unfused: time na2d_qk_rpb, na2d_softmax and na2d_av one by one instead")
     return ap.parse_args(argv)
 
 
@@ -415,6 +417,69 @@ def roofline_of(w, launch_s, kernel_kind, peaks, peak_src):
     }
 
 
+def run_unfused(args, w, dev, peaks, peak_src):
+    """Times the unfused chain call by call: na2d_qk_rpb (q, k -> float32
+    logits), na2d_softmax (in place) and na2d_av (weights, v -> out), each
+    replayed from CUDA graphs over rotating input sets larger than L2, and
+    reports per call the time, the algorithmic bytes it moves and the
+    fraction of the HBM roofline."""
+    import torch
+
+    from vision_sliding_window_b200 import na2d
+    from vision_sliding_window_b200.inputs import workload_inputs
+
+    host = workload_inputs(w)
+    es = w.elem_bytes
+    tensor = w.queries * w.d * es
+    attn_bytes = w.queries * w.ks * w.ks * 4
+    rpb_bytes = w.heads * (2 * w.ks - 1) ** 2 * es
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = max(2, math.ceil(3 * l2 / (3 * tensor + attn_bytes)))
+    sets = []
+    for _ in range(R):
+        q, k, v, rpb = (t.to(dev) for t in host)
+        sets.append((q, k, v, rpb, torch.empty((*q.shape[:4], w.ks * w.ks), device=dev), torch.empty_like(q)))
+    calls = {
+        "na2d_qk_rpb": (lambda s: na2d.qk_rpb(s[0], s[1], s[3], w.ks, attn=s[4]), 2 * tensor + attn_bytes + rpb_bytes),
+        "na2d_softmax": (lambda s: na2d.softmax_(s[4], w.ks, 1.0 / math.sqrt(w.d)), 2 * attn_bytes),
+        "na2d_av": (lambda s: na2d.av(s[4], s[2], w.ks, out=s[5]), attn_bytes + 2 * tensor),
+    }
+    steps = max(args.steps, 20)
+    res = {}
+    total_us = 0.0
+    for name, (fn, nbytes) in calls.items():
+        for i in range(max(args.warmup, 3)):
+            fn(sets[i % R])
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(steps):
+                fn(sets[i % R])
+        g.replay()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        us = e0.elapsed_time(e1) * 1e3 / steps
+        del g
+        gbs = nbytes / us / 1e3
+        total_us += us
+        res[name] = {"us_per_call": us, "algorithmic_bytes": nbytes, "gbs": gbs, "frac": gbs / peaks["hbm_gbs"]}
+    if na2d.device_status() != na2d.NA_OK:
+        raise SystemExit("device status not OK after the unfused chain")
+    line = {
+        "metric": METRIC, "api": "unfused", "value": w.query_neighbours / (total_us * 1e-6) / 1e9, "unit": UNIT,
+        "n_gpus": 1, "steps": steps, "warmup": args.warmup, "ms_per_step": total_us / 1e3,
+        "higher_is_better": True, "dtype": w.dtype, "data": "synthetic",
+        "config": workload_config(w, 1, {"l2": f"rotating {R} sets", "timing": "CUDA graphs, CUDA events"}),
+        "calls": res, "peak_source": peak_src, "gpu_launches": 3 * steps,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     from vision_sliding_window_b200.dist import barrier, env_rank, max_over_ranks
@@ -438,6 +503,10 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     na2d.load_library()
     peaks, peak_src = load_peaks()
+    if args.api == "unfused":
+        if world > 1:
+            raise SystemExit("--api unfused runs on one GPU")
+        return run_unfused(args, w, dev, peaks, peak_src)
 
     sampler = ClockSampler(local_rank) if rank == 0 else None
     if sampler:
